@@ -1,0 +1,356 @@
+#!/usr/bin/env python
+"""SSD forward throughput on one B200 per rank (tokens/s = batch * seqlen / s).
+
+Default workload: the 2.7B-like layer (B4 L8192 H80 P64 N128 G1, chunk 256, bf16
+inputs). One step = one ssd_fwd call over one batch of seeded synthetic inputs
+that already sit in HBM. Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU: launch with torch.distributed.run; every rank runs its own batch
+(weak scaling, no data-path collective; the process group only carries the
+barrier and the max over ranks of the device time).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SSD fwd tokens/s (batch·seqlen/s) at 2.7B-layer shape; % of roofline"
+UNIT = "tokens/s"
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d["hbm_gbs"], d["bf16_tflops"], "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def algorithmic(wl):
+    """Bytes each input is read once + outputs written once; FLOPs of the chunked
+    method with the structurally-zero upper triangle of the diagonal blocks skipped
+    and C B^T counted once per (batch, chunk, group)."""
+    B, L, H, P, N, G, Q = wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.dstate, wl.ngroups, wl.chunk
+    e = 2 if wl.dtype == "bf16" else 4
+    nbytes = (2 * B * L * H * P * e       # x in, y out
+              + B * L * H * e             # dt
+              + 2 * B * L * G * N * e     # B, C
+              + 2 * H * 4                 # A, D
+              + B * H * P * N * 4         # h_final
+              + (B * H * P * N * 4 if wl.h0_std > 0 else 0))
+    nc_full, tail = divmod(L, Q)
+    tri = lambda q: q * (q + 1) / 2
+    pairs = nc_full * tri(Q) + tri(tail)      # causal (l, s) pairs per (b, head-or-group)
+    flops = B * (2 * pairs * N * G + 2 * pairs * P * H) + B * L * H * 4 * P * N
+    return nbytes, flops
+
+
+class ClockSampler:
+    """nvidia-smi samples (SM clock, throttle reasons) while the timed region runs."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        rows = [r.split(", ") for r in open(self.file.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons, util = [], 0.0, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                s, mx, u = float(r[2]), float(r[3]), float(r[5])
+            except (ValueError, IndexError):
+                continue
+            smax = max(smax, mx)
+            util.append(u)
+            if u > 0:
+                sm.append(s)
+                for nm, v in zip(names, r[7:11]):
+                    if v.strip().lower() == "active":
+                        reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax or None,
+                "reasons": sorted(reasons), "samples": len(rows), "samples_busy": len(sm)}
+
+
+def dist_setup():
+    import torch
+    import torch.distributed as dist
+
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def reduce_max(v: float, ws: int) -> float:
+    if ws == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle timing (the CPU baseline and the reference arm)
+
+def time_oracle(wl, d, target_s: float):
+    """Run the fp64 oracle on whole (b, h) streams (every token of the sequence) of
+    the drawn inputs, as many streams as fit in about target_s. Returns (tokens/s
+    extrapolated to the whole problem, streams run, threads, seconds)."""
+    import oracle
+
+    threads = os.cpu_count() or 1
+    B, H = wl.batch, wl.nheads
+
+    def run(nb, nh):
+        G = wl.ngroups
+        hpg = H // G
+        if G > 1:  # keep whole groups so the head -> group map is unchanged
+            nh = max(hpg, (nh // hpg) * hpg)
+        ng = nh // hpg if G > 1 else 1
+        hs, gs = (slice(0, nb), slice(None), slice(0, nh)), (slice(0, nb), slice(None), slice(0, ng))
+        x, dt = d["x"].values(hs), d["dt"].values(hs)
+        Bm, Cm = d["B"].values(gs), d["C"].values(gs)
+        A, D = d["A"].value[:nh], d["D"].value[:nh]
+        h0 = d["h0"].values((slice(0, nb), slice(0, nh))) if d["h0"] is not None else None
+        t0 = time.perf_counter()
+        oracle.recurrent(x, dt, A, Bm, Cm, D, h0, threads=threads)
+        return time.perf_counter() - t0, nb * nh
+
+    t1, n1 = run(1, 1)
+    want = max(1, int(target_s / max(t1, 1e-6) * threads))
+    nb = min(B, max(1, want // H)) if want >= H else 1
+    nh = H if want >= H else min(H, want)
+    t, n = run(nb, nh)
+    tokens = wl.batch * wl.seqlen
+    value = tokens * n / (B * H) / t
+    return value, n, threads, t
+
+
+def reference_arm(args, wl):
+    """The CPU oracle as the reference arm, on the same workload and metric."""
+    from state_space_sequence_chunked_b200 import inputs
+
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    d = inputs.draw(wl)
+    per_step = max(1.0, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
+    vals, secs = [], []
+    for i in range(args.warmup + args.steps):
+        v, n, threads, t = time_oracle(wl, d, per_step)
+        if i >= args.warmup:
+            vals.append(v)
+            secs.append(t)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * wl.batch * wl.seqlen / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "seqlen": wl.seqlen, "nheads": wl.nheads,
+                   "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"fp64 recurrence on {n} of {wl.batch * wl.nheads} (batch, head) streams "
+                                   f"over all {wl.seqlen} tokens per step, extrapolated to the whole batch"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mamba2_2p7b")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    from state_space_sequence_chunked_b200 import inputs
+
+    wl = inputs.WORKLOADS[args.workload]
+    if wl.verify:
+        raise SystemExit("bench.py times the forward workloads")
+    if args.impl == "reference":
+        return reference_arm(args, wl)
+
+    import torch
+
+    from state_space_sequence_chunked_b200 import _binding as ssd
+
+    ws, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    d = inputs.draw(wl, seed=wl.seed + 1000 * rank)
+    code = ssd.SSD_BF16 if wl.dtype == "bf16" else ssd.SSD_F32
+    plan = ssd.fwd_plan(wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.ngroups, wl.dstate, code, wl.chunk)
+    g = {k: d[k].torch(dev) for k in ("x", "dt", "A", "B", "C", "D")}
+    h0 = d["h0"].torch(dev) if d["h0"] is not None else None
+    y = torch.empty_like(g["x"])
+    hf = torch.empty(wl.batch, wl.nheads, wl.headdim, wl.dstate, device=dev)
+    work = torch.empty(max(plan["workspace_bytes"], 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ssd.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], h0, chunk=wl.chunk, y=y, h_final=hf,
+                    workspace=work, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.2)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms_max = reduce_max(ms, ws)
+
+    tokens = wl.batch * wl.seqlen
+    value = tokens * ws / (ms_max * 1e-3)
+    hbm, tf, src = peaks()
+    nbytes, flops = algorithmic(wl)
+    t_roof = max(nbytes / (hbm * 1e9), flops / (tf * 1e12))
+    bound = "hbm" if nbytes / (hbm * 1e9) >= flops / (tf * 1e12) else "tensor"
+    if bound == "hbm":
+        achieved, peak, unit = nbytes / (ms * 1e-3) / 1e9, hbm, "GB/s"
+    else:
+        achieved, peak, unit = flops / (ms * 1e-3) / 1e12, tf, "TFLOP/s"
+
+    # end to end through the public call with host buffers
+    host = {k: v.cpu().pin_memory() for k, v in g.items()}
+    h0_host = h0.cpu().pin_memory() if h0 is not None else None
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    hf_host = torch.empty(hf.shape, dtype=hf.dtype).pin_memory()
+    dg = {k: torch.empty_like(v) for k, v in g.items()}
+    dh0 = torch.empty_like(h0) if h0 is not None else None
+
+    def e2e_step():
+        for k in dg:
+            dg[k].copy_(host[k], non_blocking=True)
+        if dh0 is not None:
+            dh0.copy_(h0_host, non_blocking=True)
+        ssd.ssd_fwd(dg["x"], dg["dt"], dg["A"], dg["B"], dg["C"], dg["D"], dh0, chunk=wl.chunk, y=y,
+                    h_final=hf, workspace=work, stream=stream)
+        y_host.copy_(y, non_blocking=True)
+        hf_host.copy_(hf, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    e2e_ms = reduce_max(ev0.elapsed_time(ev1) / e2e_steps, ws)
+    h2d = sum(v.numel() * v.element_size() for v in host.values()) + (
+        h0_host.numel() * 4 if h0_host is not None else 0)
+    d2h = y_host.numel() * y_host.element_size() + hf_host.numel() * 4
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        v, n, threads, t = time_oracle(wl, d, args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"fp64 recurrence on {n} of {wl.batch * wl.nheads} (batch, head) streams over all "
+                         f"{wl.seqlen} tokens ({t:.1f} s), extrapolated to the whole batch"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "seqlen": wl.seqlen, "nheads": wl.nheads,
+                       "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk,
+                       "path": plan["path"], "per_rank_batch": wl.batch,
+                       "l2": "inputs larger than L2 (x and y 335.5 MB each per step vs 126 MB L2); no flush"},
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                         "frac": achieved / peak, "traffic": None,
+                         "kernel": "whole ssd_fwd call (%d launches)" % plan["kernels"],
+                         "peak_source": src, "alg_bytes": nbytes, "alg_flops": flops,
+                         "roofline_tokens_per_s": tokens / t_roof, "frac_of_roofline_time": t_roof / (ms * 1e-3)},
+            "cpu_baseline": cpu,
+            "e2e": {"value": tokens * ws / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": plan["kernels"] * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

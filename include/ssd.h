@@ -1,0 +1,151 @@
+/*
+ * libssd: the Mamba-2 SSD (state space duality) layer forward pass on B200
+ * (sm_100a), evaluated with the chunked algorithm, and its speculative-decoding
+ * verify step.
+ *
+ * Per batch row b and head h (group g = h / (nheads / ngroups)):
+ *     h_t = exp(dt_t * A_h) * h_{t-1} + dt_t * x_t B_t^T      (P x N state)
+ *     y_t = h_t C_t + D_h * x_t
+ * Sources: Mamba-2 SSD write-up (msbhsh.com), sections "SSD 层" (the SSD layer:
+ * a selective SSM whose A is a scalar per head) and "SSD 算法：分块和状态传递"
+ * (chunks of Q tokens; intra-chunk matmuls, chunk states, a short scan across
+ * chunks, state-to-output); "A Visual Guide to Mamba and SSMs", "What is a SSM"
+ * (D is a skip connection) and "The Recurrent Representation"; the Llama-to-Mamba
+ * distillation write-up, "推测解码" (verify K draft tokens, keep the state at the
+ * accepted position).
+ *
+ * Conventions for every entry point below:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, row-major and
+ *    contiguous, 16-byte aligned. The library allocates no memory, keeps no global
+ *    mutable state and may be called from several host threads at once.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream). Calls are asynchronous: SSD_OK means "validated and launched".
+ *    Faults inside a kernel surface from a later CUDA call or synchronisation.
+ *  - Arguments are validated before anything is launched; on an error status no
+ *    kernel was launched and no output was touched. Nothing aborts or prints.
+ *  - x, dt, B, C and y share one storage type (ssd_dtype_t). A, D, h0, h_final,
+ *    states_out and h_keep are always fp32. Arithmetic is fp32 (accumulation in
+ *    fp32; bf16 products on tensor cores where the inputs are bf16).
+ *  - The head-to-group map is contiguous: head h reads group h / (nheads/ngroups).
+ */
+#ifndef SSD_H
+#define SSD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct ssd_shape_t {
+    int64_t batch;   /* B >= 0 */
+    int64_t seqlen;  /* L >= 0 (for ssd_verify: the number of draft tokens K) */
+    int64_t nheads;  /* H >= 1 */
+    int64_t headdim; /* P, 1..256 */
+    int64_t ngroups; /* G >= 1, divides H */
+    int64_t dstate;  /* N, 1..256 */
+} ssd_shape_t;
+
+typedef enum ssd_dtype_t {
+    SSD_F32 = 0,  /* IEEE fp32 */
+    SSD_BF16 = 1, /* bfloat16; y is rounded to nearest even from fp32 */
+} ssd_dtype_t;
+
+typedef enum ssd_status_t {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1, /* NULL required pointer, negative or inconsistent size */
+    SSD_ERR_UNSUPPORTED = 2, /* a size outside the supported range */
+    SSD_ERR_ALIGNMENT = 3,   /* a pointer not 16-byte aligned */
+    SSD_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required */
+    SSD_ERR_CUDA = 5,        /* a CUDA runtime call failed (launch or attribute) */
+    SSD_ERR_TIMEOUT = 6,     /* a bounded device-side wait ran out */
+} ssd_status_t;
+
+/* Human-readable text for a status code (static storage, never NULL). */
+const char *ssd_strerror(ssd_status_t status);
+
+/* The implementation ssd_fwd selects for a problem (see ssd_fwd_plan). */
+typedef enum ssd_path_t {
+    SSD_PATH_NONE = 0,    /* nothing to compute (batch == 0 or seqlen == 0) */
+    SSD_PATH_SIMT = 1,    /* chunked, fp32 CUDA-core arithmetic, one kernel per step */
+    SSD_PATH_TCGEN05 = 2, /* chunked, fused, bf16 tcgen05 tensor-core MMAs */
+} ssd_path_t;
+
+typedef struct ssd_plan_t {
+    int32_t path;           /* an ssd_path_t */
+    int32_t kernels;        /* kernel launches per ssd_fwd call */
+    size_t workspace_bytes; /* same value as ssd_fwd_workspace_bytes */
+} ssd_plan_t;
+
+/*
+ * Describe what ssd_fwd would launch for this problem, without launching.
+ * Errors: as ssd_fwd_workspace_bytes; *plan is untouched on error.
+ */
+ssd_status_t ssd_fwd_plan(const ssd_shape_t *shape, ssd_dtype_t dtype, int64_t chunk,
+                          ssd_plan_t *plan);
+
+/*
+ * Bytes of device workspace that ssd_fwd needs for this problem
+ * (written to *bytes; 0 is possible). The per-chunk intermediates (within-chunk
+ * decay cumsums and, on some paths, chunk states) live there.
+ * Errors: SSD_ERR_INVALID_ARG / SSD_ERR_UNSUPPORTED as ssd_fwd would return.
+ */
+ssd_status_t ssd_fwd_workspace_bytes(const ssd_shape_t *shape, ssd_dtype_t dtype, int64_t chunk,
+                                     size_t *bytes);
+
+/*
+ * SSD forward pass over a whole sequence, by the chunked algorithm with chunk
+ * size `chunk` (1..256; the last chunk may be shorter).
+ *   x        [B, L, H, P]   dtype          input (the "V" of the attention view)
+ *   dt       [B, L, H]      dtype          step size, used as given (no softplus)
+ *   A        [H]            fp32           decay rate per head (A_h <= 0 expected)
+ *   Bm, Cm   [B, L, G, N]   dtype          input and output projections
+ *   D        [H]            fp32 or NULL   skip weight (NULL = 0)
+ *   h0       [B, H, P, N]   fp32 or NULL   initial state (NULL = zeros)
+ *   y        [B, L, H, P]   dtype          output
+ *   h_final  [B, H, P, N]   fp32 or NULL   state after the last token
+ *   workspace, workspace_bytes             >= ssd_fwd_workspace_bytes(...)
+ * seqlen == 0 writes only h_final (= h0 or zeros); batch == 0 does nothing.
+ */
+ssd_status_t ssd_fwd(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *x, const void *dt,
+                     const float *A, const void *Bm, const void *Cm, const float *D,
+                     const float *h0, int64_t chunk, void *y, float *h_final, void *workspace,
+                     size_t workspace_bytes, void *stream);
+
+/*
+ * Speculative-decoding verify: run K draft tokens from the saved state h0 and
+ * return every intermediate state, so the caller can keep the state at the
+ * position where verification stops. shape->seqlen must equal K (1..64).
+ *   h0          [B, H, P, N]      fp32           state before the first draft token
+ *   x           [B, K, H, P]      dtype
+ *   dt          [B, K, H]         dtype
+ *   A, D        [H]               fp32 (D may be NULL = 0)
+ *   Bm, Cm      [B, K, G, N]      dtype
+ *   states_out  [B, K, H, P, N]   fp32           state after draft token k
+ *   y           [B, K, H, P]      dtype          outputs of the K tokens
+ * Requires dstate % 4 == 0.
+ */
+ssd_status_t ssd_verify(const ssd_shape_t *shape, ssd_dtype_t dtype, const float *h0,
+                        const void *x, const void *dt, const float *A, const void *Bm,
+                        const void *Cm, const float *D, int64_t K, float *states_out, void *y,
+                        void *stream);
+
+/*
+ * Keep the state at the accepted position, once the caller has decided how many
+ * draft tokens of each batch row were accepted:
+ *   h_keep[b] = h0[b]                       if accepted[b] == 0
+ *             = states_out[b, accepted[b]-1] if 1 <= accepted[b] <= K
+ * A bit-exact copy. `accepted` is a device int32 array [B]. A row whose index is
+ * outside 0..K is filled with quiet NaN (the host cannot see device values).
+ * shape->seqlen is ignored; dims as in ssd_verify.
+ */
+ssd_status_t ssd_select_state(const ssd_shape_t *shape, int64_t K, const float *h0,
+                              const float *states_out, const int32_t *accepted, float *h_keep,
+                              void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_H */

@@ -1,0 +1,169 @@
+"""ctypes binding of libssd (include/ssd.h): argument marshalling only.
+
+Every step of the computation runs in the CUDA library. Torch tensors supply
+device memory and the current CUDA stream. If the library is missing the calls
+raise; there is no other implementation behind them.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libssd.so")
+
+SSD_F32, SSD_BF16 = 0, 1
+STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "SSD_ERR_ALIGNMENT",
+          4: "SSD_ERR_WORKSPACE", 5: "SSD_ERR_CUDA", 6: "SSD_ERR_TIMEOUT"}
+
+
+class SSDError(RuntimeError):
+    def __init__(self, status: int, fn: str, text: str):
+        super().__init__(f"{fn}: {STATUS.get(status, status)} ({text})")
+        self.status = status
+        self.name = STATUS.get(status, str(status))
+
+
+class ShapeT(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("batch", "seqlen", "nheads", "headdim", "ngroups", "dstate")]
+
+
+class PlanT(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int32), ("kernels", ctypes.c_int32), ("workspace_bytes", ctypes.c_size_t)]
+
+
+PATHS = {0: "none", 1: "simt", 2: "tcgen05"}
+
+_lib = None
+_vp, _i64, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+_SIGS = {
+    "ssd_strerror": ([ctypes.c_int], ctypes.c_char_p),
+    "ssd_fwd_workspace_bytes": ([ctypes.POINTER(ShapeT), ctypes.c_int, _i64, ctypes.POINTER(_sz)], ctypes.c_int),
+    "ssd_fwd_plan": ([ctypes.POINTER(ShapeT), ctypes.c_int, _i64, ctypes.POINTER(PlanT)], ctypes.c_int),
+    "ssd_fwd": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 7 + [_i64, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "ssd_verify": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 7 + [_i64, _vp, _vp, _vp], ctypes.c_int),
+    "ssd_select_state": ([ctypes.POINTER(ShapeT), _i64] + [_vp] * 5, ctypes.c_int),
+}
+
+
+def lib():
+    """Load libssd.so (built in-tree by state_space_sequence_chunked_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libssd.so is not built ({LIB_PATH}); run state_space_sequence_chunked_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            f = getattr(L, name)
+            f.argtypes, f.restype = args, res
+        _lib = L
+    return _lib
+
+
+def _check(status: int, fn: str):
+    if status != 0:
+        raise SSDError(status, fn, lib().ssd_strerror(status).decode())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SSD_F32
+    if t.dtype == torch.bfloat16:
+        return SSD_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dev(*ts):
+    dev = None
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("libssd takes CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError("libssd takes contiguous tensors")
+        dev = t.device if dev is None else dev
+    return dev
+
+
+def _stream(dev, stream):
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def fwd_workspace_bytes(batch, seqlen, nheads, headdim, ngroups, dstate, dtype_code, chunk) -> int:
+    shape = ShapeT(batch, seqlen, nheads, headdim, ngroups, dstate)
+    out = _sz(0)
+    _check(lib().ssd_fwd_workspace_bytes(ctypes.byref(shape), dtype_code, chunk, ctypes.byref(out)),
+           "ssd_fwd_workspace_bytes")
+    return out.value
+
+
+def fwd_plan(batch, seqlen, nheads, headdim, ngroups, dstate, dtype_code, chunk) -> dict:
+    """{'path': 'simt'|'tcgen05'|'none', 'kernels': launches per call, 'workspace_bytes': int}."""
+    shape = ShapeT(batch, seqlen, nheads, headdim, ngroups, dstate)
+    out = PlanT()
+    _check(lib().ssd_fwd_plan(ctypes.byref(shape), dtype_code, chunk, ctypes.byref(out)), "ssd_fwd_plan")
+    return {"path": PATHS.get(out.path, str(out.path)), "kernels": out.kernels,
+            "workspace_bytes": out.workspace_bytes}
+
+
+def ssd_fwd(x, dt, A, B, C, D=None, h0=None, *, chunk: int, y=None, h_final=None,
+            return_final_state: bool = True, workspace=None, stream=None):
+    """y, h_final = ssd_fwd(x [B,L,H,P], dt [B,L,H], A [H] f32, B/C [B,L,G,N], D [H] f32?, h0 [B,H,P,N] f32?)."""
+    dev = _dev(x, dt, A, B, C, D, h0, y, h_final, workspace)
+    Bsz, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    code = _dtype_code(x)
+    shape = ShapeT(Bsz, L, H, P, G, N)
+    if y is None:
+        y = torch.empty_like(x)
+    if h_final is None and return_final_state:
+        h_final = torch.empty((Bsz, H, P, N), dtype=torch.float32, device=dev)
+    need = fwd_workspace_bytes(Bsz, L, H, P, G, N, code, chunk)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().ssd_fwd(ctypes.byref(shape), code, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                       _ptr(h0), chunk, _ptr(y), _ptr(h_final), _ptr(workspace), ws_bytes,
+                       _stream(dev, stream))
+    _check(st, "ssd_fwd")
+    return y, h_final
+
+
+def ssd_verify(h0, x, dt, A, B, C, D=None, *, states_out=None, y=None, stream=None):
+    """y [B,K,H,P], states_out [B,K,H,P,N] = ssd_verify(h0 [B,H,P,N] f32, x [B,K,H,P], dt, A, B, C, D)."""
+    dev = _dev(h0, x, dt, A, B, C, D, states_out, y)
+    Bsz, K, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    shape = ShapeT(Bsz, K, H, P, G, N)
+    if y is None:
+        y = torch.empty_like(x)
+    if states_out is None:
+        states_out = torch.empty((Bsz, K, H, P, N), dtype=torch.float32, device=dev)
+    st = lib().ssd_verify(ctypes.byref(shape), _dtype_code(x), _ptr(h0), _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
+                          _ptr(C), _ptr(D), K, _ptr(states_out), _ptr(y), _stream(dev, stream))
+    _check(st, "ssd_verify")
+    return y, states_out
+
+
+def ssd_select_state(h0, states_out, accepted, *, h_keep=None, stream=None):
+    """h_keep[b] = h0[b] if accepted[b] == 0 else states_out[b, accepted[b] - 1] (bit-exact)."""
+    dev = _dev(h0, states_out, accepted, h_keep)
+    Bsz, K, H, P, N = states_out.shape
+    if accepted.dtype != torch.int32:
+        raise TypeError("accepted must be int32")
+    shape = ShapeT(Bsz, K, H, P, 1, N)
+    if h_keep is None:
+        h_keep = torch.empty_like(h0)
+    st = lib().ssd_select_state(ctypes.byref(shape), K, _ptr(h0), _ptr(states_out), _ptr(accepted),
+                                _ptr(h_keep), _stream(dev, stream))
+    _check(st, "ssd_select_state")
+    return h_keep

@@ -1,0 +1,170 @@
+// The C ABI: argument validation, workspace sizing and path selection.
+// Every check runs before any launch; on an error nothing is launched.
+#include "ssd_internal.cuh"
+
+#define SSD_API extern "C" __attribute__((visibility("default")))
+
+namespace ssd {
+namespace {
+
+constexpr int64_t kMaxDim = 256;      // headdim, dstate
+constexpr int64_t kMaxChunk = 256;
+constexpr int64_t kMaxGridYZ = 65535; // batch and nheads map to grid y/z
+constexpr int64_t kMaxVerifyK = 64;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ssd_status_t check_shape(const ssd_shape_t *s) {
+    if (!s) return SSD_ERR_INVALID_ARG;
+    if (s->batch < 0 || s->seqlen < 0 || s->nheads < 1 || s->headdim < 1 || s->ngroups < 1 ||
+        s->dstate < 1)
+        return SSD_ERR_INVALID_ARG;
+    if (s->nheads % s->ngroups != 0) return SSD_ERR_INVALID_ARG;
+    if (s->headdim > kMaxDim || s->dstate > kMaxDim) return SSD_ERR_UNSUPPORTED;
+    if (s->batch > kMaxGridYZ || s->nheads > kMaxGridYZ) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+ssd_status_t check_dtype(ssd_dtype_t d) {
+    return (d == SSD_F32 || d == SSD_BF16) ? SSD_OK : SSD_ERR_INVALID_ARG;
+}
+
+ssd_status_t make_fwd(const ssd_shape_t *s, ssd_dtype_t dtype, int64_t chunk, FwdProblem *p) {
+    ssd_status_t st = check_shape(s);
+    if (st != SSD_OK) return st;
+    if ((st = check_dtype(dtype)) != SSD_OK) return st;
+    if (chunk < 1) return SSD_ERR_INVALID_ARG;
+    if (chunk > kMaxChunk) return SSD_ERR_UNSUPPORTED;
+    *p = FwdProblem{};
+    p->B = s->batch;
+    p->L = s->seqlen;
+    p->H = s->nheads;
+    p->P = s->headdim;
+    p->G = s->ngroups;
+    p->N = s->dstate;
+    p->Q = chunk;
+    p->nc = (s->seqlen + chunk - 1) / chunk;
+    p->dtype = dtype;
+    return SSD_OK;
+}
+
+ssd_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
+
+}  // namespace
+}  // namespace ssd
+
+using namespace ssd;
+
+SSD_API const char *ssd_strerror(ssd_status_t s) {
+    switch (s) {
+    case SSD_OK: return "success";
+    case SSD_ERR_INVALID_ARG: return "invalid argument (NULL pointer, negative or inconsistent size)";
+    case SSD_ERR_UNSUPPORTED: return "unsupported size (outside the supported range)";
+    case SSD_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case SSD_ERR_WORKSPACE: return "workspace missing or too small";
+    case SSD_ERR_CUDA: return "CUDA runtime error";
+    case SSD_ERR_TIMEOUT: return "bounded device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+SSD_API ssd_status_t ssd_fwd_workspace_bytes(const ssd_shape_t *shape, ssd_dtype_t dtype,
+                                             int64_t chunk, size_t *bytes) {
+    if (!bytes) return SSD_ERR_INVALID_ARG;
+    FwdProblem p;
+    const ssd_status_t st = make_fwd(shape, dtype, chunk, &p);
+    if (st != SSD_OK) return st;
+    *bytes = (p.B == 0 || p.L == 0) ? 0 : simt_fwd_workspace_bytes(p);
+    return SSD_OK;
+}
+
+SSD_API ssd_status_t ssd_fwd_plan(const ssd_shape_t *shape, ssd_dtype_t dtype, int64_t chunk,
+                                  ssd_plan_t *plan) {
+    if (!plan) return SSD_ERR_INVALID_ARG;
+    FwdProblem p;
+    const ssd_status_t st = make_fwd(shape, dtype, chunk, &p);
+    if (st != SSD_OK) return st;
+    ssd_plan_t out{};
+    if (p.B == 0 || p.L == 0) {
+        out.path = SSD_PATH_NONE;
+        out.kernels = 0;
+        out.workspace_bytes = 0;
+    } else {
+        out.path = SSD_PATH_SIMT;
+        out.kernels = 4;
+        out.workspace_bytes = simt_fwd_workspace_bytes(p);
+    }
+    *plan = out;
+    return SSD_OK;
+}
+
+SSD_API ssd_status_t ssd_fwd(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *x,
+                             const void *dt, const float *A, const void *Bm, const void *Cm,
+                             const float *D, const float *h0, int64_t chunk, void *y,
+                             float *h_final, void *workspace, size_t workspace_bytes,
+                             void *stream) {
+    FwdProblem p;
+    ssd_status_t st = make_fwd(shape, dtype, chunk, &p);
+    if (st != SSD_OK) return st;
+    if (p.B == 0) return SSD_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t state_bytes = (size_t)(p.B * p.H * p.P * p.N) * sizeof(float);
+    if (p.L == 0) {
+        if (!h_final) return SSD_OK;
+        if (!aligned16(h_final) || (h0 && !aligned16(h0))) return SSD_ERR_ALIGNMENT;
+        return from_cuda(h0 ? cudaMemcpyAsync(h_final, h0, state_bytes, cudaMemcpyDeviceToDevice, s)
+                            : cudaMemsetAsync(h_final, 0, state_bytes, s));
+    }
+    if (!x || !dt || !A || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, dt, A, Bm, Cm, D, h0, y, h_final, workspace};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return SSD_ERR_ALIGNMENT;
+    const size_t need = simt_fwd_workspace_bytes(p);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return SSD_ERR_WORKSPACE;
+    p.x = x;
+    p.dt = dt;
+    p.A = A;
+    p.Bm = Bm;
+    p.Cm = Cm;
+    p.D = D;
+    p.h0 = h0;
+    p.y = y;
+    p.h_final = h_final;
+    return from_cuda(simt_fwd(p, workspace, s));
+}
+
+SSD_API ssd_status_t ssd_verify(const ssd_shape_t *shape, ssd_dtype_t dtype, const float *h0,
+                                const void *x, const void *dt, const float *A, const void *Bm,
+                                const void *Cm, const float *D, int64_t K, float *states_out,
+                                void *y, void *stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if ((st = check_dtype(dtype)) != SSD_OK) return st;
+    if (K < 1 || shape->seqlen != K) return SSD_ERR_INVALID_ARG;
+    if (K > kMaxVerifyK || shape->dstate % 4 != 0) return SSD_ERR_UNSUPPORTED;
+    if (shape->batch == 0) return SSD_OK;
+    if (!h0 || !x || !dt || !A || !Bm || !Cm || !states_out || !y) return SSD_ERR_INVALID_ARG;
+    const void *ptrs[] = {h0, x, dt, A, Bm, Cm, D, states_out, y};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return SSD_ERR_ALIGNMENT;
+    VerifyProblem p{shape->batch, K, shape->nheads, shape->headdim, shape->ngroups, shape->dstate,
+                    dtype, h0, x, dt, Bm, Cm, A, D, states_out, y};
+    return from_cuda(verify_launch(p, static_cast<cudaStream_t>(stream)));
+}
+
+SSD_API ssd_status_t ssd_select_state(const ssd_shape_t *shape, int64_t K, const float *h0,
+                                      const float *states_out, const int32_t *accepted,
+                                      float *h_keep, void *stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (K < 1) return SSD_ERR_INVALID_ARG;
+    if (K > kMaxVerifyK || shape->dstate % 4 != 0) return SSD_ERR_UNSUPPORTED;
+    if (shape->batch == 0) return SSD_OK;
+    if (!h0 || !states_out || !accepted || !h_keep) return SSD_ERR_INVALID_ARG;
+    const void *ptrs[] = {h0, states_out, accepted, h_keep};
+    for (const void *q : ptrs)
+        if (!aligned16(q)) return SSD_ERR_ALIGNMENT;
+    const int64_t per_row = shape->nheads * shape->headdim * shape->dstate;
+    return from_cuda(select_launch(shape->batch, K, per_row, h0, states_out, accepted, h_keep,
+                                   static_cast<cudaStream_t>(stream)));
+}

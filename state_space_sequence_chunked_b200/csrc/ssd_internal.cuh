@@ -1,0 +1,51 @@
+// Internal declarations shared by the libssd translation units (not part of the ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ssd.h"
+
+namespace ssd {
+
+// One forward problem, validated by the API layer.
+struct FwdProblem {
+    int64_t B, L, H, P, G, N, Q, nc;
+    ssd_dtype_t dtype;
+    const void *x, *dt, *Bm, *Cm;
+    const float *A, *D, *h0;
+    void *y;
+    float *h_final;
+};
+
+struct VerifyProblem {
+    int64_t B, K, H, P, G, N;
+    ssd_dtype_t dtype;
+    const float *h0;
+    const void *x, *dt, *Bm, *Cm;
+    const float *A, *D;
+    float *states_out;
+    void *y;
+};
+
+constexpr size_t kWsAlign = 256;
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ---- chunked path with fp32 CUDA-core arithmetic (exact path for fp32 inputs) ----
+size_t simt_fwd_workspace_bytes(const FwdProblem &p);
+cudaError_t simt_fwd(const FwdProblem &p, void *ws, cudaStream_t s);
+
+// ---- verify / select --------------------------------------------------------------
+cudaError_t verify_launch(const VerifyProblem &p, cudaStream_t s);
+cudaError_t select_launch(int64_t B, int64_t K, int64_t per_row, const float *h0,
+                          const float *states_out, const int32_t *accepted, float *h_keep,
+                          cudaStream_t s);
+
+// ---- element access ---------------------------------------------------------------
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ void store_as(float *p, float v) { *p = v; }
+__device__ __forceinline__ void store_as(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+
+}  // namespace ssd

@@ -1,0 +1,144 @@
+// Speculative-decoding verify and state selection.
+//
+// Verify runs K draft tokens of the recurrence from a saved state and writes the
+// state after every token (the Llama-to-Mamba distillation write-up, "推测解码":
+// the target model checks a run of draft tokens in one pass, and the state kept
+// is the one at the position where the check stops). With K small the chunked
+// form has nothing to amortise, so each state row is advanced token by token in
+// registers; the cost is the K state writes, a pure HBM stream.
+#include "ssd_internal.cuh"
+
+namespace ssd {
+namespace {
+
+constexpr int kVThreads = 256;
+constexpr int kMaxVec = 2;  // float4 vectors per lane per state row: N <= 256
+
+// grid (H, B). Warp w advances rows p = w, w + 8, ...; lane owns float4 vectors
+// v = lane + 32 j of the row. Shared memory: B, C (K x N), x (K x P), dt, decay (K).
+template <typename T>
+__global__ void __launch_bounds__(kVThreads)
+    k_verify(const float *__restrict__ h0, const T *__restrict__ x, const T *__restrict__ dt,
+             const float *__restrict__ A, const T *__restrict__ Bm, const T *__restrict__ Cm,
+             const float *__restrict__ D, int K, int H, int P, int G, int N,
+             float *__restrict__ states_out, T *__restrict__ y) {
+    extern __shared__ float sm[];
+    float *bsm = sm;            // [K][N]
+    float *csm = bsm + K * N;   // [K][N]
+    float *xsm = csm + K * N;   // [K][P]
+    float *dts = xsm + K * P;   // [K]
+    float *dec = dts + K;       // [K]
+    const int h = blockIdx.x, b = blockIdx.y, g = h / (H / G);
+    const int tid = threadIdx.x;
+    for (int i = tid; i < K * N; i += blockDim.x) {
+        const int k = i / N, n = i % N;
+        const int64_t off = (((int64_t)b * K + k) * G + g) * N + n;
+        bsm[i] = to_f32(Bm[off]);
+        csm[i] = to_f32(Cm[off]);
+    }
+    for (int i = tid; i < K * P; i += blockDim.x) {
+        const int k = i / P, p = i % P;
+        xsm[i] = to_f32(x[(((int64_t)b * K + k) * H + h) * P + p]);
+    }
+    for (int k = tid; k < K; k += blockDim.x) {
+        const float d = to_f32(dt[((int64_t)b * K + k) * H + h]);
+        dts[k] = d;
+        dec[k] = expf(d * A[h]);
+    }
+    __syncthreads();
+
+    const int warp = tid >> 5, lane = tid & 31;
+    const int nv = N / 4;
+    const float Dh = D ? D[h] : 0.f;
+    for (int p = warp; p < P; p += kVThreads / 32) {
+        float4 s[kMaxVec];
+        const float4 *src = reinterpret_cast<const float4 *>(h0 + (((int64_t)b * H + h) * P + p) * N);
+#pragma unroll
+        for (int j = 0; j < kMaxVec; ++j) {
+            const int v = lane + 32 * j;
+            s[j] = v < nv ? src[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        for (int k = 0; k < K; ++k) {
+            const float dk = dec[k];
+            const float xk = xsm[k * P + p];
+            const float dx = dts[k] * xk;
+            const float4 *bk = reinterpret_cast<const float4 *>(bsm + k * N);
+            const float4 *ck = reinterpret_cast<const float4 *>(csm + k * N);
+            float4 *dst = reinterpret_cast<float4 *>(states_out + ((((int64_t)b * K + k) * H + h) * P + p) * N);
+            float part = 0.f;
+#pragma unroll
+            for (int j = 0; j < kMaxVec; ++j) {
+                const int v = lane + 32 * j;
+                if (v < nv) {
+                    const float4 bb = bk[v], cc = ck[v];
+                    s[j].x = fmaf(dk, s[j].x, dx * bb.x);
+                    s[j].y = fmaf(dk, s[j].y, dx * bb.y);
+                    s[j].z = fmaf(dk, s[j].z, dx * bb.z);
+                    s[j].w = fmaf(dk, s[j].w, dx * bb.w);
+                    part = fmaf(s[j].x, cc.x, part);
+                    part = fmaf(s[j].y, cc.y, part);
+                    part = fmaf(s[j].z, cc.z, part);
+                    part = fmaf(s[j].w, cc.w, part);
+                    __stcs(dst + v, s[j]);
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+            if (lane == 0) store_as(y + (((int64_t)b * K + k) * H + h) * P + p, part + Dh * xk);
+        }
+    }
+}
+
+// grid (ceil(per_row / 4 / 256), B)
+__global__ void k_select(const float *__restrict__ h0, const float *__restrict__ so,
+                         const int32_t *__restrict__ accepted, int K, int64_t per_row,
+                         float *__restrict__ out) {
+    const int b = blockIdx.y;
+    const int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t nv = per_row / 4;
+    if (v >= nv) return;
+    const int a = accepted[b];
+    float4 *dst = reinterpret_cast<float4 *>(out + (int64_t)b * per_row);
+    if (a < 0 || a > K) {
+        const float qn = __int_as_float(0x7fc00000);
+        dst[v] = make_float4(qn, qn, qn, qn);
+        return;
+    }
+    const float *src = a == 0 ? h0 + (int64_t)b * per_row : so + ((int64_t)b * K + (a - 1)) * per_row;
+    dst[v] = reinterpret_cast<const float4 *>(src)[v];
+}
+
+}  // namespace
+
+cudaError_t verify_launch(const VerifyProblem &p, cudaStream_t s) {
+    const int K = (int)p.K, H = (int)p.H, P = (int)p.P, G = (int)p.G, N = (int)p.N;
+    const size_t smem = (size_t)(2 * K * N + K * P + 2 * K) * sizeof(float);
+    cudaError_t e;
+    dim3 grid(H, (unsigned)p.B);
+    if (p.dtype == SSD_F32) {
+        if ((e = cudaFuncSetAttribute(k_verify<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+            return e;
+        k_verify<float><<<grid, kVThreads, smem, s>>>(p.h0, (const float *)p.x, (const float *)p.dt, p.A,
+                                                      (const float *)p.Bm, (const float *)p.Cm, p.D, K, H, P,
+                                                      G, N, p.states_out, (float *)p.y);
+    } else {
+        using bf = __nv_bfloat16;
+        if ((e = cudaFuncSetAttribute(k_verify<bf>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+            return e;
+        k_verify<bf><<<grid, kVThreads, smem, s>>>(p.h0, (const bf *)p.x, (const bf *)p.dt, p.A,
+                                                   (const bf *)p.Bm, (const bf *)p.Cm, p.D, K, H, P, G, N,
+                                                   p.states_out, (bf *)p.y);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t select_launch(int64_t B, int64_t K, int64_t per_row, const float *h0,
+                          const float *states_out, const int32_t *accepted, float *h_keep,
+                          cudaStream_t s) {
+    const int64_t nv = per_row / 4;
+    dim3 grid((unsigned)((nv + 255) / 256), (unsigned)B);
+    k_select<<<grid, 256, 0, s>>>(h0, states_out, accepted, (int)K, per_row, h_keep);
+    return cudaGetLastError();
+}
+
+}  // namespace ssd

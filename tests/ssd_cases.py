@@ -1,0 +1,78 @@
+"""Shared helpers for the GPU parity tests: run the CUDA path through the binding
+on seeded inputs, and compute the oracle on the same rounded values (whole
+problem for small sizes, sampled (b, h) streams for the full-size workloads)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from state_space_sequence_chunked_b200 import _binding as ssd
+from state_space_sequence_chunked_b200 import inputs
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def rel_err(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), "non-finite values in the GPU output"
+    return float(np.max(np.abs(got - ref)) / max(np.max(np.abs(ref)), 1e-30))
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().double().numpy() if t.dtype == torch.bfloat16 else t.detach().cpu().double().numpy()
+
+
+def gpu_inputs(d, device):
+    g = {k: d[k].torch(device) for k in ("x", "dt", "A", "B", "C", "D")}
+    g["h0"] = d["h0"].torch(device) if d["h0"] is not None else None
+    return g
+
+
+def run_fwd(d, chunk, device, *, use_D=True, use_h0=True, nan_fill=True):
+    g = gpu_inputs(d, device)
+    y = torch.empty_like(g["x"])
+    hf = torch.empty(g["x"].shape[0], g["x"].shape[2], g["x"].shape[3], g["B"].shape[3], device=device)
+    if nan_fill:
+        y.fill_(float("nan"))
+        hf.fill_(float("nan"))
+    ssd.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"] if use_D else None,
+                g["h0"] if use_h0 else None, chunk=chunk, y=y, h_final=hf)
+    torch.cuda.synchronize()
+    return y, hf
+
+
+def oracle_full(d, *, use_D=True, use_h0=True):
+    h0 = d["h0"].value if (use_h0 and d["h0"] is not None) else None
+    return oracle.recurrent(d["x"].value, d["dt"].value, d["A"].value, d["B"].value, d["C"].value,
+                            d["D"].value if use_D else None, h0)
+
+
+def oracle_stream(d, b, h):
+    """Oracle y[b, :, h, :] and h_final[b, h] of one stream, from the sliced inputs."""
+    H = d["x"].shape[2]
+    G = d["B"].shape[2]
+    g = h // (H // G)
+    x = d["x"].values((slice(b, b + 1), slice(None), slice(h, h + 1)))
+    dt = d["dt"].values((slice(b, b + 1), slice(None), slice(h, h + 1)))
+    Bm = d["B"].values((slice(b, b + 1), slice(None), slice(g, g + 1)))
+    Cm = d["C"].values((slice(b, b + 1), slice(None), slice(g, g + 1)))
+    A = d["A"].value[h:h + 1]
+    D = d["D"].value[h:h + 1]
+    h0 = d["h0"].values((slice(b, b + 1), slice(h, h + 1))) if d["h0"] is not None else None
+    y, hf = oracle.recurrent(x, dt, A, Bm, Cm, D, h0)
+    return y[0, :, 0, :], hf[0, 0]
+
+
+def sample_streams(Bsz, H, n, seed=123):
+    rng = np.random.default_rng(seed)
+    picks = {(0, 0), (Bsz - 1, H - 1)}
+    while len(picks) < min(n, Bsz * H):
+        picks.add((int(rng.integers(Bsz)), int(rng.integers(H))))
+    return sorted(picks)
+
+
+def draw(name, **kw):
+    return inputs.draw(inputs.WORKLOADS[name], **kw)

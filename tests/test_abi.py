@@ -1,0 +1,126 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/*.h declares, sizes its workspace, and rejects bad arguments before it
+launches anything."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from state_space_sequence_chunked_b200 import _binding as B
+from state_space_sequence_chunked_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.lib()
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(ssd_[A-Za-z0-9_]+)\s*\(", text, re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("ssd_fwd", "ssd_verify", "ssd_select_state", "ssd_fwd_workspace_bytes", "ssd_strerror"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_strerror(lib):
+    for code in range(7):
+        assert lib.ssd_strerror(code)
+    assert lib.ssd_strerror(99) == b"unknown status"
+
+
+def ws(shape, dtype=B.SSD_BF16, chunk=256):
+    out = ctypes.c_size_t(0)
+    st = B.lib().ssd_fwd_workspace_bytes(ctypes.byref(B.ShapeT(*shape)), dtype, chunk, ctypes.byref(out))
+    return st, out.value
+
+
+def test_workspace_bytes(lib):
+    st, n = ws((4, 8192, 80, 64, 1, 128))
+    assert st == 0 and n > 0
+    st0, n0 = ws((4, 0, 80, 64, 1, 128))
+    assert st0 == 0 and n0 == 0
+    assert ws((1, 10, 4, 16, 3, 16))[0] == 1    # H % G != 0
+    assert ws((1, 10, 4, 16, 1, 16), chunk=0)[0] == 1
+    assert ws((1, 10, 4, 16, 1, 16), chunk=512)[0] == 2
+    assert ws((1, 10, 4, 512, 1, 16))[0] == 2
+    assert ws((1, 10, 4, 16, 1, 16), dtype=7)[0] == 1
+    assert lib.ssd_fwd_workspace_bytes(ctypes.byref(B.ShapeT(1, 1, 1, 1, 1, 1)), 0, 1, None) == 1
+
+
+def fwd_call(shape, ptrs, chunk=64, ws_bytes=1 << 30, dtype=B.SSD_BF16):
+    s = B.ShapeT(*shape)
+    p = {k: ctypes.c_void_p(v) if v else None for k, v in ptrs.items()}
+    return B.lib().ssd_fwd(ctypes.byref(s), dtype, p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], p["h0"],
+                           chunk, p["y"], p["hf"], p["ws"], ws_bytes, None)
+
+
+GOOD = dict(x=0x10000, dt=0x20000, A=0x30000, B=0x40000, C=0x50000, D=0x60000, h0=None, y=0x70000,
+            hf=0x80000, ws=0x90000)
+
+
+def test_fwd_rejects_before_launch(lib):
+    shape = (2, 100, 4, 16, 2, 16)
+    assert lib.ssd_fwd(None, 1, *([None] * 7), 64, None, None, None, 0, None) == 1
+    for k in ("x", "dt", "A", "B", "C", "y"):
+        assert fwd_call(shape, {**GOOD, k: None}) == 1, k
+    for k in ("x", "dt", "A", "B", "C", "D", "y", "hf", "ws"):
+        assert fwd_call(shape, {**GOOD, k: GOOD[k] + 4}) == 3, k
+    assert fwd_call(shape, {**GOOD, "ws": None}) == 4
+    assert fwd_call(shape, GOOD, ws_bytes=16) == 4
+    assert fwd_call((2, 100, 4, 16, 3, 16), GOOD) == 1
+    assert fwd_call((-1, 100, 4, 16, 1, 16), GOOD) == 1
+    assert fwd_call((2, 100, 0, 16, 1, 16), GOOD) == 1
+    assert fwd_call((2, 100, 4, 300, 1, 16), GOOD) == 2
+    assert fwd_call((2, 100, 4, 16, 1, 300), GOOD) == 2
+    assert fwd_call((70000, 100, 4, 16, 1, 16), GOOD) == 2
+    assert fwd_call(shape, GOOD, chunk=0) == 1
+    assert fwd_call(shape, GOOD, chunk=257) == 2
+    assert fwd_call(shape, GOOD, dtype=3) == 1
+    # batch == 0 is a valid empty problem: nothing to launch, nothing touched
+    assert fwd_call((0, 100, 4, 16, 1, 16), {k: None for k in GOOD}) == 0
+
+
+def test_verify_and_select_reject_before_launch(lib):
+    s = B.ShapeT(2, 8, 4, 16, 2, 16)
+    v = lambda **kw: lib.ssd_verify(ctypes.byref(kw.get("shape", s)), 1, *[ctypes.c_void_p(a) if a else None for a in kw.get(
+        "p", [0x1000] * 7)], kw.get("K", 8), ctypes.c_void_p(0x2000), ctypes.c_void_p(0x3000), None)
+    assert v(K=7) == 1                       # seqlen != K
+    assert v(K=0, shape=B.ShapeT(2, 0, 4, 16, 2, 16)) == 1
+    assert v(K=65, shape=B.ShapeT(2, 65, 4, 16, 2, 16)) == 2
+    assert v(shape=B.ShapeT(2, 8, 4, 16, 2, 18)) == 2   # dstate % 4
+    assert v(p=[0x1000, None, 0x1000, 0x1000, 0x1000, 0x1000, None]) == 1
+    assert v(p=[0x1008] + [0x1000] * 6) == 3
+    sel = lambda K=8, acc=0x4000, shape=s: lib.ssd_select_state(ctypes.byref(shape), K, ctypes.c_void_p(0x1000),
+                                                                 ctypes.c_void_p(0x2000), ctypes.c_void_p(acc) if acc else None,
+                                                                 ctypes.c_void_p(0x3000), None)
+    assert sel(K=0) == 1
+    assert sel(acc=None) == 1
+    assert sel(acc=0x4004) == 3
+    assert sel(shape=B.ShapeT(2, 8, 4, 16, 2, 6)) == 2
+
+
+def test_binding_requires_cuda_tensors():
+    import torch
+
+    x = torch.zeros(1, 4, 2, 8)
+    with pytest.raises(ValueError):
+        B.ssd_fwd(x, torch.zeros(1, 4, 2), torch.zeros(2), torch.zeros(1, 4, 1, 8), torch.zeros(1, 4, 1, 8), chunk=4)
