@@ -114,6 +114,39 @@ ssd_status_t ssd_fwd(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *x,
                      size_t workspace_bytes, void *stream);
 
 /*
+ * ssd_fwd for callers that cannot allocate device memory. No counterpart in
+ * the pages describing the method: this entry point exists for deployment.
+ *
+ * Some callers cannot call cudaMalloc: an inference server that reserves all of
+ * HBM up front and manages it itself, a real-time loop where an allocation could
+ * block or fail, a plugin whose host framework owns every allocation and passes
+ * in only input and output buffers. They cannot supply ssd_fwd's workspace.
+ * This entry point takes the same inputs and outputs as ssd_fwd, minus the
+ * workspace, and allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * call). Its intermediates live in one built-in device array of
+ * SSD_STATIC_SCRATCH_BYTES (16 MiB), which every GPU that loads the library holds
+ * until the process exits.
+ *  - Always runs the fp32 CUDA-core kernels (the exact path of ssd_fwd).
+ *  - Problems whose intermediates need more than SSD_STATIC_SCRATCH_BYTES return
+ *    SSD_ERR_WORKSPACE before launching anything (ssd_fwd_plan's workspace_bytes,
+ *    for a problem ssd_fwd runs on the CUDA-core path, is the amount needed).
+ *  - The first call on each device looks up the array's device address (with that
+ *    device current) and caches it; make that first call before any CUDA stream
+ *    capture begins.
+ *  - All calls on a device share the one array, which keeps the previous call's
+ *    contents (every element read is first written by the same call, so stale
+ *    contents are harmless). Calls that may overlap on the GPU -- on different
+ *    streams, or from several host threads without ordering -- race on it:
+ *    serialise them.
+ */
+#define SSD_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+
+ssd_status_t ssd_fwd_static_scratch(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *x,
+                                    const void *dt, const float *A, const void *Bm,
+                                    const void *Cm, const float *D, const float *h0,
+                                    int64_t chunk, void *y, float *h_final, void *stream);
+
+/*
  * Speculative-decoding verify: run K draft tokens from the saved state h0 and
  * return every intermediate state, so the caller can keep the state at the
  * position where verification stops. shape->seqlen must equal K (1..64).
