@@ -50,6 +50,24 @@ ssd_status_t make_fwd(const ssd_shape_t *s, ssd_dtype_t dtype, int64_t chunk, Fw
 
 ssd_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
 
+// Path selection: the fused tensor-core kernel where its shape constraints hold,
+// the fp32 CUDA-core kernels otherwise (fp32 inputs always take the latter).
+ssd_plan_t plan_of(const FwdProblem &p) {
+    ssd_plan_t out{};
+    if (p.B == 0 || p.L == 0) {
+        out.path = SSD_PATH_NONE;
+    } else if (tc_supported(p)) {
+        out.path = SSD_PATH_TCGEN05;
+        out.kernels = 1;
+        out.workspace_bytes = tc_fwd_workspace_bytes(p);
+    } else {
+        out.path = SSD_PATH_SIMT;
+        out.kernels = 4;
+        out.workspace_bytes = simt_fwd_workspace_bytes(p);
+    }
+    return out;
+}
+
 }  // namespace
 }  // namespace ssd
 
@@ -74,7 +92,7 @@ SSD_API ssd_status_t ssd_fwd_workspace_bytes(const ssd_shape_t *shape, ssd_dtype
     FwdProblem p;
     const ssd_status_t st = make_fwd(shape, dtype, chunk, &p);
     if (st != SSD_OK) return st;
-    *bytes = (p.B == 0 || p.L == 0) ? 0 : simt_fwd_workspace_bytes(p);
+    *bytes = plan_of(p).workspace_bytes;
     return SSD_OK;
 }
 
@@ -84,16 +102,7 @@ SSD_API ssd_status_t ssd_fwd_plan(const ssd_shape_t *shape, ssd_dtype_t dtype, i
     FwdProblem p;
     const ssd_status_t st = make_fwd(shape, dtype, chunk, &p);
     if (st != SSD_OK) return st;
-    ssd_plan_t out{};
-    if (p.B == 0 || p.L == 0) {
-        out.path = SSD_PATH_NONE;
-        out.kernels = 0;
-        out.workspace_bytes = 0;
-    } else {
-        out.path = SSD_PATH_SIMT;
-        out.kernels = 4;
-        out.workspace_bytes = simt_fwd_workspace_bytes(p);
-    }
+    const ssd_plan_t out = plan_of(p);
     *plan = out;
     return SSD_OK;
 }
@@ -119,8 +128,9 @@ SSD_API ssd_status_t ssd_fwd(const ssd_shape_t *shape, ssd_dtype_t dtype, const 
     const void *ptrs[] = {x, dt, A, Bm, Cm, D, h0, y, h_final, workspace};
     for (const void *q : ptrs)
         if (q && !aligned16(q)) return SSD_ERR_ALIGNMENT;
-    const size_t need = simt_fwd_workspace_bytes(p);
-    if (need > 0 && (!workspace || workspace_bytes < need)) return SSD_ERR_WORKSPACE;
+    const ssd_plan_t plan = plan_of(p);
+    if (plan.workspace_bytes > 0 && (!workspace || workspace_bytes < plan.workspace_bytes))
+        return SSD_ERR_WORKSPACE;
     p.x = x;
     p.dt = dt;
     p.A = A;
@@ -130,7 +140,7 @@ SSD_API ssd_status_t ssd_fwd(const ssd_shape_t *shape, ssd_dtype_t dtype, const 
     p.h0 = h0;
     p.y = y;
     p.h_final = h_final;
-    return from_cuda(simt_fwd(p, workspace, s));
+    return from_cuda(plan.path == SSD_PATH_TCGEN05 ? tc_fwd(p, workspace, s) : simt_fwd(p, workspace, s));
 }
 
 SSD_API ssd_status_t ssd_verify(const ssd_shape_t *shape, ssd_dtype_t dtype, const float *h0,

@@ -36,6 +36,11 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 size_t simt_fwd_workspace_bytes(const FwdProblem &p);
 cudaError_t simt_fwd(const FwdProblem &p, void *ws, cudaStream_t s);
 
+// ---- fused chunked path on tcgen05 tensor cores (bf16, P = 64, N in {128, 256}) ----
+bool tc_supported(const FwdProblem &p);
+size_t tc_fwd_workspace_bytes(const FwdProblem &p);
+cudaError_t tc_fwd(const FwdProblem &p, void *ws, cudaStream_t s);
+
 // ---- verify / select --------------------------------------------------------------
 cudaError_t verify_launch(const VerifyProblem &p, cudaStream_t s);
 cudaError_t select_launch(int64_t B, int64_t K, int64_t per_row, const float *h0,

@@ -31,16 +31,29 @@ def gpu_inputs(d, device):
     return g
 
 
+def plan_of(d, chunk):
+    Bsz, L, H, P = d["x"].shape
+    G, N = d["B"].shape[2], d["B"].shape[3]
+    code = ssd.SSD_BF16 if d["x"].dtype == "bf16" else ssd.SSD_F32
+    return ssd.fwd_plan(Bsz, L, H, P, G, N, code, chunk)
+
+
 def run_fwd(d, chunk, device, *, use_D=True, use_h0=True, nan_fill=True):
+    """Run ssd_fwd; also checks the device status word that the tensor-core path
+    leaves at the start of its workspace (0 = no bounded wait ran out)."""
     g = gpu_inputs(d, device)
     y = torch.empty_like(g["x"])
     hf = torch.empty(g["x"].shape[0], g["x"].shape[2], g["x"].shape[3], g["B"].shape[3], device=device)
     if nan_fill:
         y.fill_(float("nan"))
         hf.fill_(float("nan"))
+    plan = plan_of(d, chunk)
+    ws = torch.full((max(plan["workspace_bytes"], 16),), 0xAB, dtype=torch.uint8, device=device)
     ssd.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"] if use_D else None,
-                g["h0"] if use_h0 else None, chunk=chunk, y=y, h_final=hf)
+                g["h0"] if use_h0 else None, chunk=chunk, y=y, h_final=hf, workspace=ws)
     torch.cuda.synchronize()
+    if plan["path"] == "tcgen05":
+        assert int(ws[:4].view(torch.int32).item()) == 0, "device status word set"
     return y, hf
 
 

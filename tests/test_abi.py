@@ -66,6 +66,17 @@ def test_workspace_bytes(lib):
     assert lib.ssd_fwd_workspace_bytes(ctypes.byref(B.ShapeT(1, 1, 1, 1, 1, 1)), 0, 1, None) == 1
 
 
+def test_plan_selects_path(lib):
+    plan = B.fwd_plan(4, 8192, 80, 64, 1, 128, B.SSD_BF16, 256)
+    assert plan["path"] == "tcgen05" and plan["kernels"] == 1
+    assert B.fwd_plan(1, 65536, 80, 64, 1, 256, B.SSD_BF16, 256)["path"] == "tcgen05"
+    assert B.fwd_plan(1, 256, 4, 16, 1, 16, B.SSD_F32, 64)["path"] == "simt"
+    assert B.fwd_plan(4, 8192, 80, 64, 1, 128, B.SSD_F32, 256)["path"] == "simt"
+    assert B.fwd_plan(4, 8192, 80, 64, 1, 128, B.SSD_BF16, 64)["path"] == "simt"
+    assert B.fwd_plan(4, 8192, 80, 128, 1, 128, B.SSD_BF16, 256)["path"] == "simt"
+    assert B.fwd_plan(4, 0, 80, 64, 1, 128, B.SSD_BF16, 256)["path"] == "none"
+
+
 def fwd_call(shape, ptrs, chunk=64, ws_bytes=1 << 30, dtype=B.SSD_BF16):
     s = B.ShapeT(*shape)
     p = {k: ctypes.c_void_p(v) if v else None for k, v in ptrs.items()}

@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 import torch
 
-from ssd_cases import TOL, draw, oracle_full, oracle_stream, rel_err, run_fwd, sample_streams, to_np
+from ssd_cases import TOL, draw, oracle_full, oracle_stream, plan_of, rel_err, run_fwd, sample_streams, to_np
 from state_space_sequence_chunked_b200 import _binding as ssd
 from state_space_sequence_chunked_b200 import inputs
 
@@ -75,6 +75,58 @@ def test_seqlen_zero_copies_initial_state(cuda_device):
     y, hf = ssd.ssd_fwd(x, dt, A, Bm, Bm, None, None, chunk=64)
     torch.cuda.synchronize()
     assert torch.count_nonzero(hf) == 0
+
+
+@pytest.mark.parametrize("name", ["mamba2_130m", "mamba2_2p7b", "long_n256"])
+def test_bf16_workloads_take_the_tensor_core_path(name):
+    wl = inputs.WORKLOADS[name]
+    d = inputs.draw(wl, batch=1, seqlen=8)
+    assert plan_of(d, wl.chunk)["path"] == "tcgen05"
+
+
+def _tc_case(seed, **kw):
+    wl = dataclasses.replace(inputs.WORKLOADS["mamba2_130m"], batch=1, seqlen=128, nheads=1, h0_std=0.5, seed=seed)
+    return inputs.draw(dataclasses.replace(wl, **kw))
+
+
+def _zeroed(d, *names):
+    d = dict(d)
+    for n in names:
+        if n == "h0":
+            d["h0"] = None
+            continue
+        t = d[n]
+        z = object.__new__(type(t))
+        z.__dict__.update(t.__dict__)
+        z.bits = np.zeros_like(t.bits)
+        z._value = None
+        d[n] = z
+    return d
+
+
+@pytest.mark.parametrize("what", ["skip", "state_to_output", "diagonal_block", "all"])
+def test_tensor_core_products_in_isolation(cuda_device, what):
+    """One 128-token block with all but one product switched off, so a wrong
+    operand layout shows up as exactly one failing case:
+    skip: dt = 0, h0 = 0 -> y = D x;  state_to_output: dt = 0, x = 0, D = 0 -> y = C h0^T;
+    diagonal_block: h0 = 0, D = 0 -> y = (C B^T o L) (dt x), h_final = chunk state."""
+    d = _tc_case(7)
+    zero = {"skip": ("dt", "h0"), "state_to_output": ("dt", "x", "D"), "diagonal_block": ("h0", "D"),
+            "all": ()}[what]
+    d = _zeroed(d, *zero)
+    assert plan_of(d, 128)["path"] == "tcgen05"
+    check_full(d, 128, cuda_device)
+
+
+@pytest.mark.parametrize("chunk", [128, 256])
+def test_tensor_core_path_matches_cuda_core_path(cuda_device, chunk):
+    """Same inputs through both CUDA paths (chunk 64 selects the fp32 CUDA-core path)."""
+    d = _tc_case(11, batch=2, seqlen=777, nheads=4, ngroups=2, h0_std=0.2)
+    assert plan_of(d, chunk)["path"] == "tcgen05" and plan_of(d, 64)["path"] == "simt"
+    y1, h1 = run_fwd(d, chunk, cuda_device)
+    y2, h2 = run_fwd(d, 64, cuda_device)
+    assert rel_err(to_np(y1), to_np(y2)) <= 2e-2
+    assert rel_err(to_np(h1), to_np(h2)) <= 2e-2
 
 
 @pytest.mark.parametrize("name,nstreams", [("mamba2_130m", 6), ("mamba2_2p7b", 4), ("long_n256", 3)])
