@@ -1,27 +1,39 @@
 // Fused chunked SSD forward on 5th-generation tensor cores (tcgen05, sm_100a).
 //
-// One CTA owns one (batch row b, head h) stream and walks its blocks of 128 tokens
-// in order, so x is read once, y is written once and the running state never
-// leaves the SM. Per block (the four steps of "SSD 算法：分块和状态传递" in the
+// A persistent grid (one CTA per SM) splits the B*H*nc (stream, 128-token block)
+// tasks into equal contiguous shares; within a share each stream's blocks are
+// walked in order, so x is read once, y is written once and the running state
+// stays on chip. Per block (the four steps of "SSD 算法：分块和状态传递" in the
 // Mamba-2 SSD write-up, with the block decomposition of "SSD 算法：分块矩阵分解"):
 //   step 0  A_cs[l] = sum_{j<=l} dt_j A_h            (within the block, log2 domain)
 //   step 1  G = C B^T on tensor cores (TMEM), then G'[l,s] = G[l,s] exp(A_cs[l]-A_cs[s]) dt_s
-//           for s <= l (0 above the diagonal), written back to TMEM as bf16, and
-//           Y_diag = G' X on tensor cores with G' as the TMEM A operand
+//           for s <= l (0 above the diagonal) plus D_h on the diagonal, written back to
+//           TMEM as bf16, and Y_diag = G' X with G' as the TMEM A operand (this also
+//           yields the D x skip term)
 //   step 2  dS^T = B^T X' on tensor cores, X'[s,:] = exp(A_cs[127]-A_cs[s]) dt_s x_s
 //   step 3  S <- exp(A_cs[127]) S + dS                 (fp32, registers)
 //   step 4  Y_off = C S_in^T on tensor cores (S_in in bf16 shared memory), and
-//           y = Y_diag + exp(A_cs[l]) Y_off + D_h x
+//           y = Y_diag + exp(A_cs[l]) Y_off
 // A chunk argument of 256 is evaluated as two 128-token diagonal blocks; the
 // 128x128 block between them goes through the state (its low-rank factor), which
 // is the same matrix product re-associated.
 //
-// Warp roles (320 threads): warp 0 loads (TMA + dt), warp 1 owns TMEM and issues
-// every MMA from one thread, warps 2-5 ("T") do step 0, X' and G', warps 6-9
-// ("E") run the state chain and the epilogue. Every wait is bounded: on timeout
-// the CTA raises a status word in the workspace, drains its own TMA loads and
-// MMAs, frees TMEM and returns.
+// A stream whose blocks fall into two CTAs' shares is cut: the CTA holding its
+// first part runs that part first and hands the state over through global memory
+// (the state passing of the sequence-parallel scheme in the same write-up); the
+// CTA holding the rest runs it last, so the hand-over is ready long before it is
+// read. The wait for it is bounded all the same.
+//
+// Warp roles (384 threads): warp 0 loads (TMA + dt) and issues Y_diag; warps 1, 2
+// and 3 issue C B^T, the chunk states and Y_off (one issuing thread per product:
+// an MMA instruction keeps its issuing warp busy for ~100 cycles, so the products
+// are issued in parallel); warps 4-7 ("T") do step 0, G' and X'; warps 8-11 ("E")
+// run the state chain and the epilogue. Every wait is bounded: on timeout the CTA
+// raises a status word in the workspace, drains its own TMA loads and MMAs, frees
+// TMEM and returns.
 #include <cuda.h>
+
+#include <algorithm>
 
 #include "ssd_internal.cuh"
 
@@ -30,8 +42,8 @@ namespace tc {
 
 constexpr int kQ = 128;  // tokens per diagonal block
 constexpr int kP = 64;   // head dimension handled by this path
-constexpr int kThreads = 320;
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpT = 2, kWarpE = 6;
+constexpr int kThreads = 384;
+constexpr int kWarpTma = 0, kWarpG = 1, kWarpDs = 2, kWarpYs = 3, kWarpE = 8;  // warps 4-7: T
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
 
@@ -45,7 +57,6 @@ struct Cfg {
     static constexpr int kYBufs = kWide ? 1 : 2;
     static constexpr int kStBufs = kWide ? 1 : 2;
     static constexpr bool kDsInG = !kWide;
-    static constexpr bool kXInRegs = !kWide;  // epilogue keeps its x row in registers
     static constexpr int kPanels = N / 64;           // 64-column panels of B and C
     static constexpr int kPanelBytes = kQ * 128;     // 128 rows x 128 B
     static constexpr int kCBytes = kPanels * kPanelBytes;
@@ -55,11 +66,14 @@ struct Cfg {
     static constexpr int kOffXp = kStages * kStageBytes;
     static constexpr int kOffSt = kOffXp + kXBytes;
     static constexpr int kOffSmall = kOffSt + kStBufs * kStBytes;
+    // per stage: dt, A_cs (log2 domain), the two column-factor arrays of step 1 and the block total
     static constexpr int kOffDts = kOffSmall;                       // float [kStages][128]
-    static constexpr int kOffAcsT = kOffDts + kStages * kQ * 4;     // float [4 warps][128]
-    static constexpr int kOffCfT = kOffAcsT + 4 * kQ * 4;           // float [4 warps][128]
-    static constexpr int kOffBar = kOffCfT + 4 * kQ * 4;            // uint64 barriers
-    static constexpr int kNumBars = 2 * kStages + 11 + kStBufs + 2 * kYBufs;
+    static constexpr int kOffAcs = kOffDts + kStages * kQ * 4;      // float [kStages][128]
+    static constexpr int kOffCfE = kOffAcs + kStages * kQ * 4;      // float [kStages][128]
+    static constexpr int kOffCfS = kOffCfE + kStages * kQ * 4;      // float [kStages][128]
+    static constexpr int kOffTot = kOffCfS + kStages * kQ * 4;      // float [kStages][4]
+    static constexpr int kOffBar = kOffTot + kStages * 16;          // uint64 barriers
+    static constexpr int kNumBars = 2 * kStages + 13 + kStBufs + 2 * kYBufs;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;         // tmem base, abort flag
     static constexpr int kSmemBytes = kOffMisc + 16;
     static constexpr int kSmemAlloc = kSmemBytes + 1024;            // slack for 1024-B alignment
@@ -76,10 +90,33 @@ struct Params {
     const float *A, *D, *h0;
     float *h_final;
     __nv_bfloat16 *y;
-    int *status;
-    long long L;
+    int *status;         // bit 0: a bounded wait ran out
+    int *flags;          // [gridDim.x] hand-over counters (zeroed before the launch)
+    float *handover;     // [gridDim.x][P][N] state at the end of each CTA's first part
+    long long L, total;  // total = B * H * nc tasks
     int H, G, nc;
 };
+
+// The share of CTA i is [lo, hi) in (stream-major, block-minor) task order, run as
+// [B0, hi) (the start of the last stream it touches), then [A0, B0) (whole streams),
+// then [lo, A0) (the rest of a stream begun by CTA i-1).
+struct Share {
+    long long lo, hi, a0, b0;
+    __device__ __forceinline__ int count() const { return (int)(hi - lo); }
+    __device__ __forceinline__ long long task(int t) const {
+        const long long n1 = hi - b0, n2 = b0 - a0;
+        return t < n1 ? b0 + t : (t < n1 + n2 ? a0 + (t - n1) : lo + (t - n1 - n2));
+    }
+};
+__device__ __forceinline__ Share share_of(long long total, int nc, int i, int G) {
+    const long long q = total / G, r = total % G;
+    Share s;
+    s.lo = q * i + (r * i) / G;
+    s.hi = q * (i + 1) + (r * (i + 1)) / G;
+    s.a0 = min(((s.lo + nc - 1) / nc) * nc, s.hi);
+    s.b0 = max((s.hi / nc) * nc, s.a0);
+    return s;
+}
 
 // ---------------------------------------------------------------------------------
 // PTX wrappers
@@ -108,6 +145,20 @@ __device__ __forceinline__ bool mbar_try(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// As mbar_try, but a thread whose phase is not complete sleeps (up to the hint, in ns)
+// until it completes instead of returning at once, so waiting warps take no issue slots
+// from the warps that do the work.
+__device__ __forceinline__ bool mbar_try_sleep(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(0x989680u)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -132,15 +183,13 @@ __device__ __noinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile
                                         int *status) {
     if (mbar_try(bar, parity)) return true;
     const unsigned long long t0 = now_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try(bar, parity)) return true;
-        if ((i & 63u) == 0) {
-            if (*abort_flag) return false;
-            if (now_ns() - t0 > kWaitNs) {
-                *abort_flag = 1;
-                atomicOr(status, 1);
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_sleep(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (now_ns() - t0 > kWaitNs) {
+            *abort_flag = 1;
+            atomicOr(status, 1);
+            return false;
         }
     }
 }
@@ -162,6 +211,37 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, u
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
+
+// L2 policies: B and C tiles are read by every head of their group, so they should stay;
+// x is read once and y written once, so they should go first.
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void tma_load_4d_hint(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1,
+                                                 int c2, int c3, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, "
+        "%4, %5, %6}], [%2], %7;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void *src, int c0, int c1, int c2,
+                                             int c3, uint64_t policy) {
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3, %4, %5}], [%1], %6;" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (sm100 format: version 1).
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -262,29 +342,29 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volati
 // (lane handles i = lane + 32 m). v[m] is the value at index 32 m + lane; the
 // block total is returned. Every warp runs the same sequence of operations, so
 // every warp gets bit-identical values.
-__device__ __forceinline__ float warp_block_scan(const float *dts, float a2, int lane, float (&v)[4]) {
-    float carry = 0.f;
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        float x = dts[32 * m + lane] * a2;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float u = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += u;
-        }
-        x += carry;
-        v[m] = x;
-        carry = __shfl_sync(0xffffffffu, x, 31);
-    }
-    return carry;
-}
-
 // ---------------------------------------------------------------------------------
+
+// Bounded spin on a hand-over counter in global memory.
+__device__ __noinline__ bool wait_flag(const int *flag, int want, volatile int *abort_flag, int *status) {
+    const unsigned long long t0 = now_ns();
+    for (;;) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v >= want) return true;
+        if (*abort_flag) return false;
+        if (now_ns() - t0 > kWaitNs) {
+            *abort_flag = 1;
+            atomicOr(status, 1);
+            return false;
+        }
+        __nanosleep(200);
+    }
+}
 
 template <int N>
 __global__ void __launch_bounds__(kThreads, 1)
     k_ssd_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-             const __grid_constant__ CUtensorMap tm_c, const Params prm) {
+             const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y, const Params prm) {
     using Cf = Cfg<N>;
     constexpr int S = Cf::kStages, YB = Cf::kYBufs, SB = Cf::kStBufs;
     extern __shared__ unsigned char smem_raw[];
@@ -292,49 +372,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     float *dts = reinterpret_cast<float *>(sm + Cf::kOffDts);
+    float *acs_s = reinterpret_cast<float *>(sm + Cf::kOffAcs);
+    float *cfe_s = reinterpret_cast<float *>(sm + Cf::kOffCfE);
+    float *cfs_s = reinterpret_cast<float *>(sm + Cf::kOffCfS);
+    float *tot_s = reinterpret_cast<float *>(sm + Cf::kOffTot);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + Cf::kOffBar);
     uint64_t *full = bar;                // [S]   stage loaded (TMA bytes + dt)
-    uint64_t *empty = full + S;          // [S]   stage consumed (MMA commit + 4 T warps + 4 E warps)
+    uint64_t *empty = full + S;          // [S]   stage consumed: 4 issuer commits + 4 T warps + 4 E warps
     uint64_t *gfull = empty + S;         // [2]   C B^T in score buffer j
     uint64_t *gp = gfull + 2;            // [2]   G' written back to score buffer j (T)
     uint64_t *xpr = gp + 2;              // [1]   X' written (T)
-    uint64_t *dsdone = xpr + 1;          // [2]   chunk state of block c done (MMA commit), buffer c % 2
-    uint64_t *dsfree = dsdone + 2;       // [2]   chunk state of block c read by E
-    uint64_t *sready = dsfree + 2;       // [SB]  S_in^T of block c written (E)
-    uint64_t *yfull = sready + SB;       // [YB]  Y_diag and Y_off of block c done (MMA commit)
-    uint64_t *yfree = yfull + YB;        // [YB]  Y of block c read by E
-    uint64_t *fin = yfree + YB;          // [1]   every MMA of this CTA done
+    uint64_t *dsdone = xpr + 1;          // [2]   chunk state of block t done, buffer t % 2
+    uint64_t *dsfree = dsdone + 2;       // [2]   chunk state of block t read by E
+    uint64_t *ydd = dsfree + 2;          // [2]   Y_diag of block t done (score buffer t % 2 reusable)
+    uint64_t *sready = ydd + 2;          // [SB]  S_in^T of block t written (E)
+    uint64_t *yfull = sready + SB;       // [YB]  Y_diag and Y_off of block t done
+    uint64_t *yfree = yfull + YB;        // [YB]  Y of block t read by E
+    uint64_t *fin = yfree + YB;          // [1]   every MMA of this CTA done (4 issuers)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + Cf::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + Cf::kOffMisc + 4);
     int *status = prm.status;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int H = prm.H, b = blockIdx.x / H, h = blockIdx.x % H, g = h / (H / prm.G);
+    const int H = prm.H, nc = prm.nc, hpg = prm.H / prm.G;
     const long long L = prm.L;
-    const int nc = prm.nc;
+    const Share sh = share_of(prm.total, nc, blockIdx.x, gridDim.x);
+    const int ntask = sh.count();
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1 + 4 + 4);
+            mbar_init(&empty[i], 4 + 4 + 4);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&gfull[i], 1);
             mbar_init(&gp[i], 128);
             mbar_init(&dsdone[i], 1);
             mbar_init(&dsfree[i], 128);
+            mbar_init(&ydd[i], 1);
         }
         mbar_init(xpr, 128);
         for (int i = 0; i < SB; ++i) mbar_init(&sready[i], 128);
         for (int i = 0; i < YB; ++i) {
-            mbar_init(&yfull[i], 1);
+            mbar_init(&yfull[i], 2);
             mbar_init(&yfree[i], 128);
         }
-        mbar_init(fin, 1);
+        mbar_init(fin, 4);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == kWarpMma) {
+    if (warp == kWarpG) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
                      "r"(Cf::kTmCols)
@@ -351,198 +438,266 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto stage_x = [&](int k) { return sm + k * Cf::kStageBytes + 2 * Cf::kCBytes; };
     unsigned char *xp = sm + Cf::kOffXp;
     auto st_buf = [&](int i) { return sm + Cf::kOffSt + i * Cf::kStBytes; };
-    // TMEM column of the chunk state of block c
-    auto ds_col = [&](int c) -> uint32_t { return Cf::kDsInG ? 128u * (uint32_t)(c & 1) + 64u : 384u; };
+    // TMEM column of the chunk state of task t
+    auto ds_col = [&](int t) -> uint32_t { return Cf::kDsInG ? 128u * (uint32_t)(t & 1) + 64u : 384u; };
+    constexpr uint32_t kIdG = idesc(128, 128, false, false);
+    constexpr uint32_t kIdDs = idesc(128, 64, true, true);
+    constexpr uint32_t kIdY = idesc(128, 64, false, true);
 
     if (warp == kWarpTma) {
-        // ------------------------------------------------------------- loads
-        // dt of the next block is fetched into registers one block ahead.
-        float dtn[4];
-        auto fetch_dt = [&](int c) {
+        // ------------------------------------------------------------- loads + Y_diag issue
+        // Task t's stage is loaded, then Y_diag of task t-1 is issued (with one stage, Y_diag of
+        // t-1 goes first: the stage of t is released only once Y_diag of t-1 is done).
+        float dtn[4], acn[4], cen[4], csn[4], totn = 0.f;
+        const uint64_t pol_keep = policy_evict_last(), pol_stream = policy_evict_first();
+        // dt of the next task, fetched into registers one task ahead, and its step 0: the
+        // within-block cumsum of dt * A_h (log2 domain) and the column factors of step 1,
+        // cfE[s] = exp(A_end - A_s) dt_s and cfS[s] = exp(A_start - A_s) dt_s, referenced to
+        // the last and the first entry of the 32-entry sub-block of s.
+        auto fetch = [&](int t) {
+            const long long gi = sh.task(t);
+            const int sidx = (int)(gi / nc), c = (int)(gi % nc), b = sidx / H, h = sidx % H;
+            const float a2 = __ldg(prm.A + h) * kLog2e;
+            float carry = 0.f;
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
-                const long long t = (long long)c * kQ + lane + 32 * m;
-                dtn[m] = t < L ? __bfloat162float(prm.dt[((long long)b * L + t) * H + h]) : 0.f;
-            }
-        };
-        fetch_dt(0);
-        int issued = 0;
-        for (int c = 0; c < nc; ++c) {
-            const int k = c % S;
-            if (c >= S && !wait_warp(&empty[k], (uint32_t)((c / S) - 1) & 1u, abort_flag, status)) break;
-            const int t0 = c * kQ;
+                const long long tt = (long long)c * kQ + lane + 32 * m;
+                dtn[m] = tt < L ? __bfloat162float(prm.dt[((long long)b * L + tt) * H + h]) : 0.f;
+                float x = dtn[m] * a2;
 #pragma unroll
-            for (int m = 0; m < 4; ++m) dts[k * kQ + lane + 32 * m] = dtn[m];
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float u = __shfl_up_sync(0xffffffffu, x, o);
+                    if (lane >= o) x += u;
+                }
+                x += carry;
+                acn[m] = x;
+                carry = __shfl_sync(0xffffffffu, x, 31);
+                const float vbeg = __shfl_sync(0xffffffffu, x, 0);
+                cen[m] = ex2(carry - x) * dtn[m];
+                csn[m] = ex2(vbeg - x) * dtn[m];
+            }
+            totn = carry;
+        };
+        auto issue_yd = [&](int t) -> bool {  // Y_diag = G' X with G' in TMEM   (M = l, N = p, K = s)
+            const int k = t % S, j = t & 1, yb = t % YB;
+            if (!wait_warp(&gp[j], (uint32_t)(t >> 1) & 1u, abort_flag, status)) return false;
+            if (t >= YB && !wait_warp(&yfree[yb], (uint32_t)((t - YB) / YB) & 1u, abort_flag, status)) return false;
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t xa = smem_u32(stage_x(k));
+#pragma unroll
+                for (int kk = 0; kk < kQ / 16; ++kk)
+                    mma_ts(tmem + Cf::kTmY + 128 * yb, tmem + 128 * j + 8 * kk, sdesc(xa + kk * 2048, 1024, 1024),
+                           kIdY, kk > 0);
+                mma_commit(&yfull[yb]);
+                mma_commit(&ydd[j]);
+                mma_commit(&empty[k]);
+            }
+            __syncwarp();
+            return true;
+        };
+        if (ntask > 0) fetch(0);
+        int nl = 0, nyd = 0;
+        bool ok = true;
+        for (int t = 0; ok && t < ntask; ++t) {
+            const int k = t % S;
+            if (S == 1 && t >= 1) {
+                if (!(ok = issue_yd(t - 1))) break;
+                nyd = t;
+            }
+            if (t >= S && !(ok = wait_warp(&empty[k], (uint32_t)((t / S) - 1) & 1u, abort_flag, status))) break;
+            const long long gi = sh.task(t);
+            const int sidx = (int)(gi / nc), c = (int)(gi % nc), b = sidx / H, h = sidx % H;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                dts[k * kQ + lane + 32 * m] = dtn[m];
+                acs_s[k * kQ + lane + 32 * m] = acn[m];
+                cfe_s[k * kQ + lane + 32 * m] = cen[m];
+                cfs_s[k * kQ + lane + 32 * m] = csn[m];
+            }
+            if (lane == 0) tot_s[k * 4] = totn;
             __syncwarp();
             if (lane == 0) {
+                const int t0 = c * kQ, g = h / hpg;
                 mbar_arrive_tx(&full[k], Cf::kTxBytes);
                 for (int pn = 0; pn < Cf::kPanels; ++pn) {
-                    tma_load_4d(stage_c(k) + pn * Cf::kPanelBytes, &tm_c, &full[k], 64 * pn, g, t0, b);
-                    tma_load_4d(stage_b(k) + pn * Cf::kPanelBytes, &tm_b, &full[k], 64 * pn, g, t0, b);
+                    tma_load_4d_hint(stage_c(k) + pn * Cf::kPanelBytes, &tm_c, &full[k], 64 * pn, g, t0, b, pol_keep);
+                    tma_load_4d_hint(stage_b(k) + pn * Cf::kPanelBytes, &tm_b, &full[k], 64 * pn, g, t0, b, pol_keep);
                 }
-                tma_load_4d(stage_x(k), &tm_x, &full[k], 0, h, t0, b);
+                tma_load_4d_hint(stage_x(k), &tm_x, &full[k], 0, h, t0, b, pol_stream);
             }
             __syncwarp();
-            issued = c + 1;
-            if (c + 1 < nc) fetch_dt(c + 1);
+            nl = t + 1;
+            if (t + 1 < ntask) fetch(t + 1);
+            if (S > 1 && t >= 1) {
+                if (!(ok = issue_yd(t - 1))) break;
+                nyd = t;
+            }
         }
+        if (ok && ntask > 0 && issue_yd(ntask - 1)) nyd = ntask;
+        if (lane == 0) mma_commit(fin);
         // drain: loads still in flight land before the CTA exits
         if (lane == 0) {
-            for (int c = max(0, issued - S); c < issued; ++c) {
+            for (int t = max(0, nl - S); t < nl; ++t) {
                 const unsigned long long t0 = now_ns();
-                while (!mbar_try(&full[c % S], (uint32_t)(c / S) & 1u) && now_ns() - t0 < kWaitNs) {
+                while (!mbar_try(&full[t % S], (uint32_t)(t / S) & 1u) && now_ns() - t0 < kWaitNs) {
                 }
             }
         }
         __syncwarp();
-    } else if (warp == kWarpMma) {
-        // ------------------------------------------------------------- MMA issue (one thread)
-        // Each product of each block is issued as soon as its operands and its
-        // accumulator are ready (non-blocking tests), so no block waits on a later one.
+    } else if (warp == kWarpG) {
+        // ------------------------------------------------------------- G = C B^T   (M = l, N = s, K = n)
         if (lane == 0) {
-            constexpr uint32_t kIdG = idesc(128, 128, false, false);
-            constexpr uint32_t kIdDs = idesc(128, 64, true, true);
-            constexpr uint32_t kIdY = idesc(128, 64, false, true);
-            int nG = 0, nDS = 0, nYs = 0, nYd = 0, nDone = 0;
-            unsigned long long last = now_ns();
-            uint32_t spins = 0;
-            while (nDone < nc) {
-                bool prog = false;
-                // G = C B^T   (M = l, N = s, K = n)
-                if (nG < nc) {
-                    const int c = nG, k = c % S, j = c & 1;
-                    bool ok = mbar_test(&full[k], (uint32_t)(c / S) & 1u);
-                    if (ok && c >= 2) {
-                        ok = nYd > c - 2 && nDS > c - 2;
-                        if (ok && Cf::kDsInG) ok = mbar_test(&dsfree[j], (uint32_t)((c - 2) >> 1) & 1u);
-                    }
-                    if (ok) {
-                        tc_fence_after();
-                        const uint32_t ca = smem_u32(stage_c(k)), ba = smem_u32(stage_b(k));
-#pragma unroll
-                        for (int kk = 0; kk < N / 16; ++kk) {
-                            const uint32_t off = (uint32_t)((kk >> 2) * Cf::kPanelBytes + (kk & 3) * 32);
-                            mma_ss(tmem + 128 * j, sdesc(ca + off, 16, 1024), sdesc(ba + off, 16, 1024), kIdG, kk > 0);
-                        }
-                        mma_commit(&gfull[j]);
-                        ++nG;
-                        prog = true;
-                    }
-                }
-                // chunk state dS^T = B^T X'   (M = n, N = p, K = s)
-                if (nDS < nG) {
-                    const int c = nDS, k = c % S, j = c & 1;
-                    bool ok = mbar_test(xpr, (uint32_t)c & 1u);
-                    if (ok) {
-                        if (Cf::kDsInG)
-                            ok = mbar_test(&gp[j], (uint32_t)(c >> 1) & 1u);
-                        else if (c >= 1)
-                            ok = mbar_test(&dsfree[(c - 1) & 1], (uint32_t)((c - 1) >> 1) & 1u);
-                    }
-                    if (ok) {
-                        tc_fence_after();
-                        const uint32_t ba = smem_u32(stage_b(k)), xa = smem_u32(xp);
-#pragma unroll
-                        for (int hf = 0; hf < N / 128; ++hf) {
-#pragma unroll
-                            for (int kk = 0; kk < kQ / 16; ++kk)
-                                mma_ss(tmem + ds_col(c) + 64 * hf,
-                                       sdesc(ba + 2 * hf * Cf::kPanelBytes + kk * 2048, Cf::kPanelBytes, 1024),
-                                       sdesc(xa + kk * 2048, Cf::kPanelBytes, 1024), kIdDs, kk > 0);
-                        }
-                        mma_commit(&dsdone[j]);
-                        ++nDS;
-                        prog = true;
-                    }
-                }
-                // Y_off = C S_in^T   (M = l, N = p, K = n)
-                if (nYs < nG) {
-                    const int c = nYs, k = c % S, yb = c % YB;
-                    bool ok = mbar_test(&sready[c % SB], (uint32_t)(c / SB) & 1u);
-                    if (ok && c >= YB) ok = mbar_test(&yfree[yb], (uint32_t)((c - YB) / YB) & 1u);
-                    if (ok) {
-                        tc_fence_after();
-                        const uint32_t ca = smem_u32(stage_c(k)), sa = smem_u32(st_buf(c % SB));
-#pragma unroll
-                        for (int kk = 0; kk < N / 16; ++kk) {
-                            const uint32_t off = (uint32_t)((kk >> 2) * Cf::kPanelBytes + (kk & 3) * 32);
-                            mma_ss(tmem + Cf::kTmY + 128 * yb + 64, sdesc(ca + off, 16, 1024),
-                                   sdesc(sa + kk * 2048, 1024, 1024), kIdY, kk > 0);
-                        }
-                        ++nYs;
-                        prog = true;
-                    }
-                }
-                // Y_diag = G' X with G' in TMEM   (M = l, N = p, K = s)
-                if (nYd < nG) {
-                    const int c = nYd, k = c % S, j = c & 1, yb = c % YB;
-                    bool ok = mbar_test(&gp[j], (uint32_t)(c >> 1) & 1u);
-                    if (ok && c >= YB) ok = mbar_test(&yfree[yb], (uint32_t)((c - YB) / YB) & 1u);
-                    if (ok) {
-                        tc_fence_after();
-                        const uint32_t xa = smem_u32(stage_x(k));
-#pragma unroll
-                        for (int kk = 0; kk < kQ / 16; ++kk)
-                            mma_ts(tmem + Cf::kTmY + 128 * yb, tmem + 128 * j + 8 * kk,
-                                   sdesc(xa + kk * 2048, 1024, 1024), kIdY, kk > 0);
-                        ++nYd;
-                        prog = true;
-                    }
-                }
-                // a block whose four products are all issued: signal its Y and release its stage
-                if (nDone < nDS && nDone < nYs && nDone < nYd) {
-                    mma_commit(&yfull[nDone % YB]);
-                    mma_commit(&empty[nDone % S]);
-                    ++nDone;
-                    prog = true;
-                }
-                if (prog) {
-                    spins = 0;
-                } else if ((++spins & 255u) == 0) {
-                    const unsigned long long t = now_ns();
-                    if (spins == 256) last = t;
-                    if (*abort_flag) break;
-                    if (t - last > kWaitNs) {
-                        *abort_flag = 1;
-                        atomicOr(status, 1);
+            for (int t = 0; t < ntask; ++t) {
+                const int k = t % S, j = t & 1;
+                if (!wait_phase(&full[k], (uint32_t)(t / S) & 1u, abort_flag, status)) break;
+                if (t >= 2) {  // score buffer j: G' of task t-2 consumed, its chunk state read
+                    if (!wait_phase(&ydd[j], (uint32_t)((t - 2) >> 1) & 1u, abort_flag, status)) break;
+                    if (Cf::kDsInG && !wait_phase(&dsfree[j], (uint32_t)((t - 2) >> 1) & 1u, abort_flag, status))
                         break;
-                    }
                 }
+                tc_fence_after();
+                const uint32_t ca = smem_u32(stage_c(k)), ba = smem_u32(stage_b(k));
+#pragma unroll
+                for (int kk = 0; kk < N / 16; ++kk) {
+                    const uint32_t off = (uint32_t)((kk >> 2) * Cf::kPanelBytes + (kk & 3) * 32);
+                    mma_ss(tmem + 128 * j, sdesc(ca + off, 16, 1024), sdesc(ba + off, 16, 1024), kIdG, kk > 0);
+                }
+                mma_commit(&gfull[j]);
+                mma_commit(&empty[k]);
             }
-            // every MMA issued by this thread completes before TMEM is released
             mma_commit(fin);
-            const unsigned long long t0 = now_ns();
-            while (!mbar_try(fin, 0) && now_ns() - t0 < kWaitNs) {
+        }
+        __syncwarp();
+    } else if (warp == kWarpDs) {
+        // ------------------------------------------------------------- dS^T = B^T X'   (M = n, N = p, K = s)
+        if (lane == 0) {
+            for (int t = 0; t < ntask; ++t) {
+                const int k = t % S, j = t & 1;
+                if (!wait_phase(xpr, (uint32_t)t & 1u, abort_flag, status)) break;
+                if (Cf::kDsInG) {  // T is done reading C B^T from the half this state goes to
+                    if (!wait_phase(&gp[j], (uint32_t)(t >> 1) & 1u, abort_flag, status)) break;
+                } else if (t >= 1) {
+                    if (!wait_phase(&dsfree[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u, abort_flag, status)) break;
+                }
+                tc_fence_after();
+                const uint32_t ba = smem_u32(stage_b(k)), xa = smem_u32(xp);
+#pragma unroll
+                for (int hf = 0; hf < N / 128; ++hf) {
+#pragma unroll
+                    for (int kk = 0; kk < kQ / 16; ++kk)
+                        mma_ss(tmem + ds_col(t) + 64 * hf,
+                               sdesc(ba + 2 * hf * Cf::kPanelBytes + kk * 2048, Cf::kPanelBytes, 1024),
+                               sdesc(xa + kk * 2048, Cf::kPanelBytes, 1024), kIdDs, kk > 0);
+                }
+                mma_commit(&dsdone[j]);
+                mma_commit(&empty[k]);
             }
+            mma_commit(fin);
+        }
+        __syncwarp();
+    } else if (warp == kWarpYs) {
+        // ------------------------------------------------------------- Y_off = C S_in^T   (M = l, N = p, K = n)
+        if (lane == 0) {
+            for (int t = 0; t < ntask; ++t) {
+                const int k = t % S, yb = t % YB;
+                if (!wait_phase(&sready[t % SB], (uint32_t)(t / SB) & 1u, abort_flag, status)) break;
+                if (!wait_phase(&full[k], (uint32_t)(t / S) & 1u, abort_flag, status)) break;
+                if (t >= YB && !wait_phase(&yfree[yb], (uint32_t)((t - YB) / YB) & 1u, abort_flag, status)) break;
+                tc_fence_after();
+                const uint32_t ca = smem_u32(stage_c(k)), sa = smem_u32(st_buf(t % SB));
+#pragma unroll
+                for (int kk = 0; kk < N / 16; ++kk) {
+                    const uint32_t off = (uint32_t)((kk >> 2) * Cf::kPanelBytes + (kk & 3) * 32);
+                    mma_ss(tmem + Cf::kTmY + 128 * yb + 64, sdesc(ca + off, 16, 1024), sdesc(sa + kk * 2048, 1024, 1024),
+                           kIdY, kk > 0);
+                }
+                mma_commit(&yfull[yb]);
+                mma_commit(&empty[k]);
+            }
+            mma_commit(fin);
         }
         __syncwarp();
     } else if (warp < kWarpE) {
-        // ------------------------------------------------------------- T: step 0, X', G'
-        const int qtr = warp & 3;  // TMEM lane quarter of this warp
+        // ------------------------------------------------------------- T: step 0, G', X'
+        const int qtr = warp & 3;  // TMEM lane quarter of this warp: rows 32 qtr .. 32 qtr + 31
         const int row = (qtr << 5) | lane;
-        float *acsW = reinterpret_cast<float *>(sm + Cf::kOffAcsT) + (warp - kWarpT) * kQ;
-        float *cfW = reinterpret_cast<float *>(sm + Cf::kOffCfT) + (warp - kWarpT) * kQ;
-        const float a2 = prm.A[h] * kLog2e;
         const uint32_t lane_off = (uint32_t)(qtr * 32) << 16;
-        for (int c = 0; c < nc; ++c) {
-            const int k = c % S, j = c & 1;
-            if (!wait_warp(&full[k], (uint32_t)(c / S) & 1u, abort_flag, status)) break;
+        for (int t = 0; t < ntask; ++t) {
+            const int k = t % S, j = t & 1;
+            const int h = (int)((sh.task(t) / nc) % H);
+            const float Dh = prm.D ? __ldg(prm.D + h) : 0.f;
+            if (!wait_warp(&full[k], (uint32_t)(t / S) & 1u, abort_flag, status)) break;
             const float *dk = dts + k * kQ;
-            float v[4];
-            const float tot = warp_block_scan(dk, a2, lane, v);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float vend = __shfl_sync(0xffffffffu, v[m], 31);  // A_cs at the end of 32-block m
-                acsW[32 * m + lane] = v[m];
-                cfW[32 * m + lane] = ex2(vend - v[m]) * dk[32 * m + lane];
-            }
-            __syncwarp();
+            const float *acsW = acs_s + k * kQ;
+            const float *cfE = cfe_s + k * kQ;
+            const float *cfS = cfs_s + k * kQ;
+            const float tot = tot_s[k * 4];
             const float acs_r = acsW[row];
-            const float dt_r = dk[row];
-            // X' (the previous block's chunk-state MMA must be done reading X')
-            if (c > 0 && !wait_warp(&dsdone[(c - 1) & 1], (uint32_t)((c - 1) >> 1) & 1u, abort_flag, status)) break;
+            const float acs_q0 = acsW[32 * qtr];
+            const float span_q = acs_q0 - acsW[32 * qtr + 31];
+            // G' = (C B^T) o decay o dt (+ D on the diagonal), in place in TMEM as packed bf16 pairs
+            if (!wait_warp(&gfull[j], (uint32_t)(t >> 1) & 1u, abort_flag, status)) break;
+            tc_fence_after();
             {
-                const float w = ex2(tot - acs_r) * dt_r;
+                const uint32_t gaddr = tmem + 128 * j + lane_off;
+                // factors of the diagonal sub-block stay inside fp32 range when its decay span is
+                // below 2^120; otherwise every element takes its own exponential
+                const bool diag_factored = span_q < 120.f;  // warp-uniform
+                const float rf_diag = ex2(acs_r - acs_q0);
+#pragma unroll 1
+                for (int jb = 0; jb < 4; ++jb) {
+                    uint32_t out[16];
+                    if (jb > qtr) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) out[i] = 0u;
+                    } else {
+                        uint32_t r[32];
+                        tmem_ld32(gaddr + 32 * jb, r);
+                        tmem_wait_ld();
+                        if (jb < qtr) {
+                            const float rf = ex2(acs_r - acsW[32 * jb + 31]);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const float2 cf = *reinterpret_cast<const float2 *>(cfE + 32 * jb + 2 * i);
+                                out[i] = pack_bf16(__uint_as_float(r[2 * i]) * rf * cf.x,
+                                                   __uint_as_float(r[2 * i + 1]) * rf * cf.y);
+                            }
+                        } else if (diag_factored) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const int s = 32 * jb + 2 * i;
+                                const float2 cf = *reinterpret_cast<const float2 *>(cfS + s);
+                                float v0 = s <= row ? __uint_as_float(r[2 * i]) * rf_diag * cf.x : 0.f;
+                                float v1 = s + 1 <= row ? __uint_as_float(r[2 * i + 1]) * rf_diag * cf.y : 0.f;
+                                v0 += s == row ? Dh : 0.f;
+                                v1 += s + 1 == row ? Dh : 0.f;
+                                out[i] = pack_bf16(v0, v1);
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const int s = 32 * jb + 2 * i;
+                                float v0 = s <= row ? __uint_as_float(r[2 * i]) * ex2(acs_r - acsW[s]) * dk[s] : 0.f;
+                                float v1 =
+                                    s + 1 <= row ? __uint_as_float(r[2 * i + 1]) * ex2(acs_r - acsW[s + 1]) * dk[s + 1]
+                                                 : 0.f;
+                                v0 += s == row ? Dh : 0.f;
+                                v1 += s + 1 == row ? Dh : 0.f;
+                                out[i] = pack_bf16(v0, v1);
+                            }
+                        }
+                    }
+                    tmem_st16(gaddr + 16 * jb, out);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&gp[j]);
+            }
+            // X' (the previous task's chunk-state MMA must be done reading X')
+            if (t > 0 && !wait_warp(&dsdone[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u, abort_flag, status)) break;
+            {
+                const float w = ex2(tot - acs_r) * dk[row];
                 const unsigned char *xs = stage_x(k);
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
@@ -557,47 +712,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_proxy_async();
                 mbar_arrive(xpr);
             }
-            // G' = (C B^T) o decay o dt, in place in TMEM as packed bf16 pairs
-            if (!wait_warp(&gfull[j], (uint32_t)(c >> 1) & 1u, abort_flag, status)) break;
-            tc_fence_after();
-            const uint32_t gaddr = tmem + 128 * j + lane_off;
-#pragma unroll 1
-            for (int jb = 0; jb < 4; ++jb) {
-                uint32_t out[16];
-                if (jb > qtr) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) out[i] = 0u;
-                } else {
-                    uint32_t r[32];
-                    tmem_ld32(gaddr + 32 * jb, r);
-                    tmem_wait_ld();
-                    if (jb < qtr) {
-                        // strictly below the diagonal sub-block: exp(A_l - A_e) * [exp(A_e - A_s) dt_s]
-                        const float rf = ex2(acs_r - acsW[32 * jb + 31]);
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int s = 32 * jb + 2 * i;
-                            out[i] = pack_bf16(__uint_as_float(r[2 * i]) * rf * cfW[s],
-                                               __uint_as_float(r[2 * i + 1]) * rf * cfW[s + 1]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int s = 32 * jb + 2 * i;
-                            const float v0 =
-                                s <= row ? __uint_as_float(r[2 * i]) * ex2(acs_r - acsW[s]) * dk[s] : 0.f;
-                            const float v1 =
-                                s + 1 <= row ? __uint_as_float(r[2 * i + 1]) * ex2(acs_r - acsW[s + 1]) * dk[s + 1]
-                                             : 0.f;
-                            out[i] = pack_bf16(v0, v1);
-                        }
-                    }
-                }
-                tmem_st16(gaddr + 16 * jb, out);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&gp[j]);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[k]);  // this warp is done with X and dt of the stage
         }
@@ -605,18 +719,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------- E: state chain + epilogue
         const int qtr = warp & 3;
         const int row = (qtr << 5) | lane;
-        const float a2 = prm.A[h] * kLog2e;
-        const float Dh = prm.D ? prm.D[h] : 0.f;
         const uint32_t lane_off = (uint32_t)(qtr * 32) << 16;
         constexpr int NH = N / 128;  // state rows per thread: n = row + 128 i
         float Sr[NH][kP];
-        const long long sbase = ((long long)b * H + h) * kP * N;
-#pragma unroll
-        for (int i = 0; i < NH; ++i)
-#pragma unroll
-            for (int p = 0; p < kP; ++p) Sr[i][p] = prm.h0 ? prm.h0[sbase + (long long)p * N + row + 128 * i] : 0.f;
-        auto write_st = [&](int c) {  // S_in^T of block c, bf16, into its buffer
-            unsigned char *stb = st_buf(c % SB);
+        auto write_st = [&](int t) {  // S_in^T of task t, bf16, into its buffer
+            unsigned char *stb = st_buf(t % SB);
+            // the buffer doubles as this warp's y staging slice: its last y store must have read it
+            if (lane == 0) bulk_wait_read();
+            __syncwarp();
 #pragma unroll
             for (int i = 0; i < NH; ++i) {
                 const int n = row + 128 * i;
@@ -631,25 +741,69 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             fence_proxy_async();
-            mbar_arrive(&sready[c % SB]);
+            mbar_arrive(&sready[t % SB]);
         };
-        write_st(0);
-        bool ok = true;
-        for (int c = 0; c < nc; ++c) {
-            const int k = c % S, j = c & 1, yb = c % YB;
-            if (!(ok = wait_warp(&full[k], (uint32_t)(c / S) & 1u, abort_flag, status))) break;
-            float v[4];
-            const float tot = warp_block_scan(dts + k * kQ, a2, lane, v);
-            const float acs_r = v[qtr];
-            uint4 xr[8];  // this thread's x row (kept only when the stage is released early)
-            if (Cf::kXInRegs) {
+        // Initial state of the piece that starts at task t: h0 (or zeros) at the start of a
+        // stream, otherwise the state handed over by the previous CTA.
+        auto load_init = [&](int t) -> bool {
+            const long long gi = sh.task(t);
+            const int sidx = (int)(gi / nc), c = (int)(gi % nc);
+            if (c == 0) {
+                const long long base = (long long)sidx * kP * N;
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) xr[ch] = *reinterpret_cast<const uint4 *>(stage_x(k) + swz(row, ch));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[k]);
+                for (int i = 0; i < NH; ++i)
+#pragma unroll
+                    for (int p = 0; p < kP; ++p)
+                        Sr[i][p] = prm.h0 ? prm.h0[base + (long long)p * N + row + 128 * i] : 0.f;
+                return true;
             }
+            if (!wait_flag(prm.flags + blockIdx.x - 1, 128, abort_flag, status)) return false;
+            const float *src = prm.handover + (long long)(blockIdx.x - 1) * kP * N;
+#pragma unroll
+            for (int i = 0; i < NH; ++i)
+#pragma unroll
+                for (int p = 0; p < kP; ++p) Sr[i][p] = __ldcg(src + p * N + row + 128 * i);
+            return true;
+        };
+        // End of a piece: the final state of the stream, or the hand-over to the next CTA.
+        auto store_final = [&](int t) {
+            const long long gi = sh.task(t);
+            const int sidx = (int)(gi / nc), c = (int)(gi % nc);
+            if (c == nc - 1) {
+                if (prm.h_final) {
+                    const long long base = (long long)sidx * kP * N;
+#pragma unroll
+                    for (int i = 0; i < NH; ++i)
+#pragma unroll
+                        for (int p = 0; p < kP; ++p) prm.h_final[base + (long long)p * N + row + 128 * i] = Sr[i][p];
+                }
+            } else {
+                float *dst = prm.handover + (long long)blockIdx.x * kP * N;
+#pragma unroll
+                for (int i = 0; i < NH; ++i)
+#pragma unroll
+                    for (int p = 0; p < kP; ++p) __stcg(dst + p * N + row + 128 * i, Sr[i][p]);
+                __threadfence();
+                atomicAdd(prm.flags + blockIdx.x, 1);
+            }
+        };
+        auto piece_end = [&](int t) {  // task t is the last of its piece in this CTA's order
+            const long long gi = sh.task(t);
+            return (int)(gi % nc) == nc - 1 || gi == sh.hi - 1;
+        };
+        bool ok = ntask > 0 && load_init(0);
+        if (ok) write_st(0);
+        for (int t = 0; ok && t < ntask; ++t) {
+            const int k = t % S, j = t & 1, yb = t % YB;
+            const long long gi = sh.task(t);
+            const int h = (int)((gi / nc) % H), c = (int)(gi % nc);
+            if (!(ok = wait_warp(&full[k], (uint32_t)(t / S) & 1u, abort_flag, status))) break;
+            const float tot = tot_s[k * 4];
+            const float acs_r = acs_s[k * kQ + row];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[k]);  // done with the step-0 values of the stage
             // step 3: S <- exp(A_cs[end]) S + dS
-            if (!(ok = wait_warp(&dsdone[j], (uint32_t)(c >> 1) & 1u, abort_flag, status))) break;
+            if (!(ok = wait_warp(&dsdone[j], (uint32_t)(t >> 1) & 1u, abort_flag, status))) break;
             tc_fence_after();
             {
                 const float gam = ex2(tot);
@@ -658,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         uint32_t r[32];
-                        tmem_ld32(tmem + ds_col(c) + 64 * i + 32 * half + lane_off, r);
+                        tmem_ld32(tmem + ds_col(t) + 64 * i + 32 * half + lane_off, r);
                         tmem_wait_ld();
 #pragma unroll
                         for (int q = 0; q < 32; ++q)
@@ -668,58 +822,70 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 mbar_arrive(&dsfree[j]);
             }
-            // with two S^T buffers the next one was last read by block c-1 (done: see epilogue c-1)
-            if (SB == 2 && c + 1 < nc) write_st(c + 1);
-            // epilogue: y = Y_diag + exp(A_cs[l]) Y_off + D x
-            if (!(ok = wait_warp(&yfull[yb], (uint32_t)(c / YB) & 1u, abort_flag, status))) break;
+            const bool last_of_piece = piece_end(t);
+            if (last_of_piece) store_final(t);
+            // S_in^T of the next task. With two buffers the one it goes to was last read by
+            // Y_off of task t-1, which is done (the epilogue of t-1 waited for it).
+            if (SB == 2 && t + 1 < ntask) {
+                if (last_of_piece && !(ok = load_init(t + 1))) break;
+                write_st(t + 1);
+            }
+            // epilogue: y = Y_diag + exp(A_cs[l]) Y_off   (D x is inside Y_diag)
+            if (!(ok = wait_warp(&yfull[yb], (uint32_t)(t / YB) & 1u, abort_flag, status))) break;
             tc_fence_after();
             {
+                // y rows of this warp (32 tokens x 64 values) are staged, 128-byte swizzled, in its
+                // 4 KB slice of the S^T buffer of task t (free: Y_off of task t is done) and written
+                // by one bulk tensor store.
                 const float el = ex2(acs_r);
-                const long long t = (long long)c * kQ + row;
-                __nv_bfloat16 *yrow = prm.y + (((long long)b * L + t) * H + h) * kP;
+                unsigned char *stage_y = st_buf(t % SB);
                 const uint32_t ya = tmem + Cf::kTmY + 128 * yb + lane_off;
 #pragma unroll
-                for (int qq = 0; qq < 8; ++qq) {  // 8 columns at a time
-                    uint32_t yd[8], ys[8];
-                    tmem_ld8(ya + 8 * qq, yd);
-                    tmem_ld8(ya + 64 + 8 * qq, ys);
+                for (int qq = 0; qq < 4; ++qq) {  // 16 columns at a time
+                    uint32_t yd[16], ys[16];
+                    tmem_ld16(ya + 16 * qq, yd);
+                    tmem_ld16(ya + 64 + 16 * qq, ys);
                     tmem_wait_ld();
-                    if (qq == 7) {
+                    if (qq == 3) {
                         tc_fence_before();
                         mbar_arrive(&yfree[yb]);
                     }
-                    const uint4 xv = Cf::kXInRegs ? xr[qq] : *reinterpret_cast<const uint4 *>(stage_x(k) + swz(row, qq));
-                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                    uint32_t o[4];
+                    uint32_t o[8];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float y0 = __uint_as_float(yd[2 * e]) + el * __uint_as_float(ys[2 * e]) + Dh * bf16_lo(xw[e]);
-                        const float y1 =
-                            __uint_as_float(yd[2 * e + 1]) + el * __uint_as_float(ys[2 * e + 1]) + Dh * bf16_hi(xw[e]);
-                        o[e] = pack_bf16(y0, y1);
-                    }
-                    if (t < L) *reinterpret_cast<uint4 *>(yrow + 8 * qq) = make_uint4(o[0], o[1], o[2], o[3]);
+                    for (int e = 0; e < 8; ++e)
+                        o[e] = pack_bf16(fmaf(el, __uint_as_float(ys[2 * e]), __uint_as_float(yd[2 * e])),
+                                         fmaf(el, __uint_as_float(ys[2 * e + 1]), __uint_as_float(yd[2 * e + 1])));
+                    *reinterpret_cast<uint4 *>(stage_y + swz(row, 2 * qq)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4 *>(stage_y + swz(row, 2 * qq + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+                }
+                fence_proxy_async();
+                __syncwarp();
+                const int r0 = c * kQ + 32 * qtr;
+                if (lane == 0 && r0 < L) {
+                    const int b = (int)(gi / nc) / H;
+                    tma_store_4d(&tm_y, stage_y + 32 * qtr * 128, 0, h, r0, b, policy_evict_first());
+                    bulk_commit();
                 }
             }
-            if (!Cf::kXInRegs) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[k]);
+            // with one S^T buffer it is free only now (Y_off of task t is done)
+            if (SB == 1 && t + 1 < ntask) {
+                if (last_of_piece && !(ok = load_init(t + 1))) break;
+                write_st(t + 1);
             }
-            // with one S^T buffer it is free only now (Y_off of block c is done)
-            if (SB == 1 && c + 1 < nc) write_st(c + 1);
-        }
-        if (ok && prm.h_final) {
-#pragma unroll
-            for (int i = 0; i < NH; ++i)
-#pragma unroll
-                for (int p = 0; p < kP; ++p) prm.h_final[sbase + (long long)p * N + row + 128 * i] = Sr[i][p];
         }
     }
 
+    if (warp >= kWarpE && lane == 0) bulk_wait_all();  // y stores have read their staging slices
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == kWarpMma) {
+    if (warp == kWarpG) {
+        if (lane == 0) {  // every issued MMA has completed before TMEM is released
+            const unsigned long long t0 = now_ns();
+            while (!mbar_try(fin, 0) && now_ns() - t0 < kWaitNs) {
+            }
+        }
+        __syncwarp();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(Cf::kTmCols)
                      : "memory");
     }
@@ -744,25 +910,32 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [B, L, X, inner] bf16 tensor, box {64, 1, 128, 1}, 128-byte swizzle.
-bool encode_4d(CUtensorMap *m, const void *base, int64_t inner, int64_t X, int64_t L, int64_t B) {
+// [B, L, X, inner] bf16 tensor, box {64, 1, rows, 1}, 128-byte swizzle.
+bool encode_4d(CUtensorMap *m, const void *base, int64_t inner, int64_t X, int64_t L, int64_t B, int rows = kQ) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)X, (cuuint64_t)L, (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)(inner * 2), (cuuint64_t)(X * inner * 2),
                                    (cuuint64_t)(L * X * inner * 2)};
-    const cuuint32_t box[4] = {64, 1, (cuuint32_t)kQ, 1};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
 template <int N>
-cudaError_t launch(const FwdProblem &p, int *status, cudaStream_t s) {
-    CUtensorMap tx, tb, tcm;
+cudaError_t launch(const FwdProblem &p, int *status, int *flags, float *handover, int grid, cudaStream_t s) {
+    CUtensorMap tx, tb, tcm, ty;
     if (!encode_4d(&tx, p.x, kP, p.H, p.L, p.B) || !encode_4d(&tb, p.Bm, N, p.G, p.L, p.B) ||
-        !encode_4d(&tcm, p.Cm, N, p.G, p.L, p.B))
+        !encode_4d(&tcm, p.Cm, N, p.G, p.L, p.B) || !encode_4d(&ty, p.y, kP, p.H, p.L, p.B, 32))
         return cudaErrorInvalidValue;
     Params prm;
     prm.dt = static_cast<const __nv_bfloat16 *>(p.dt);
@@ -772,14 +945,28 @@ cudaError_t launch(const FwdProblem &p, int *status, cudaStream_t s) {
     prm.h_final = p.h_final;
     prm.y = static_cast<__nv_bfloat16 *>(p.y);
     prm.status = status;
+    prm.flags = flags;
+    prm.handover = handover;
     prm.L = p.L;
     prm.H = (int)p.H;
     prm.G = (int)p.G;
     prm.nc = (int)((p.L + kQ - 1) / kQ);
+    prm.total = p.B * p.H * (long long)prm.nc;
     cudaError_t e = cudaFuncSetAttribute(k_ssd_tc<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<N>::kSmemAlloc);
     if (e != cudaSuccess) return e;
-    k_ssd_tc<N><<<(unsigned)(p.B * p.H), kThreads, Cfg<N>::kSmemAlloc, s>>>(tx, tb, tcm, prm);
-    return cudaGetLastError();
+    // All CTAs must be resident together (a CTA may wait for the state its neighbour hands
+    // over), which a cooperative launch guarantees.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = Cfg<N>::kSmemAlloc;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_ssd_tc<N>, tx, tb, tcm, ty, prm);
 }
 
 }  // namespace tc
@@ -789,13 +976,31 @@ bool tc_supported(const FwdProblem &p) {
            p.L >= 1 && p.L < (1ll << 31) && p.B * p.H < (1ll << 31);
 }
 
-size_t tc_fwd_workspace_bytes(const FwdProblem &) { return kWsAlign; }
+// Workspace: [status int | pad][flags int x grid | pad][hand-over states fp32 grid x P x N]
+// With at least as many streams as SMs every CTA's share covers a whole stream or more,
+// so a cut stream spans exactly two CTAs and the part that waits never waits on a part
+// that waits itself. With fewer streams each CTA takes one whole stream.
+static int tc_grid(const FwdProblem &p) {
+    const int sms = tc::num_sms() > 0 ? tc::num_sms() : 148;
+    const long long streams = p.B * p.H;
+    return (int)std::max(1ll, streams >= sms ? (long long)sms : streams);
+}
+
+size_t tc_fwd_workspace_bytes(const FwdProblem &p) {
+    const size_t g = (size_t)tc_grid(p);
+    return kWsAlign + align_up(g * sizeof(int), kWsAlign) + g * (size_t)(tc::kP * p.N) * sizeof(float);
+}
 
 cudaError_t tc_fwd(const FwdProblem &p, void *ws, cudaStream_t s) {
-    int *status = static_cast<int *>(ws);
-    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+    const int grid = tc_grid(p);
+    char *base = static_cast<char *>(ws);
+    int *status = reinterpret_cast<int *>(base);
+    int *flags = reinterpret_cast<int *>(base + kWsAlign);
+    float *handover = reinterpret_cast<float *>(base + kWsAlign + align_up((size_t)grid * sizeof(int), kWsAlign));
+    cudaError_t e = cudaMemsetAsync(base, 0, kWsAlign + (size_t)grid * sizeof(int), s);
     if (e != cudaSuccess) return e;
-    return p.N == 128 ? tc::launch<128>(p, status, s) : tc::launch<256>(p, status, s);
+    return p.N == 128 ? tc::launch<128>(p, status, flags, handover, grid, s)
+                      : tc::launch<256>(p, status, flags, handover, grid, s);
 }
 
 }  // namespace ssd
