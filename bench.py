@@ -57,54 +57,70 @@ def algorithmic(wl):
 
 
 class ClockSampler:
-    """nvidia-smi samples (SM clock, throttle reasons) while the timed region runs."""
+    """SM clock and clock-event (throttle) reasons of this rank's GPU, read through NVML
+    (the library nvidia-smi reports from) every 2 ms on a host thread; only samples
+    taken inside the timed window [mark_start, mark_end] count."""
 
-    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.file = None
+    def __init__(self, device):
+        import threading
+
+        self.samples, self.error, self.handle = [], None, None
+        self.t0 = self.t1 = None
+        self.stop_ev = threading.Event()
+        self.thread = None
+        try:
+            import pynvml as nv
+            import torch
+
+            nv.nvmlInit()
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.nv = nv
+            self.handle = nv.nvmlDeviceGetHandleByUUID(uuid)
+            self.smax = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM)
+            self.thread = threading.Thread(target=self._run, daemon=True)
+        except Exception as e:  # no NVML on this host: the line says so
+            self.error = f"{type(e).__name__}: {e}"
+
+    def _run(self):
+        nv, h = self.nv, self.handle
+        while not self.stop_ev.is_set():
+            t = time.perf_counter()
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((t, sm, rs))
+            except Exception as e:
+                self.error = f"{type(e).__name__}: {e}"
+                return
+            time.sleep(0.002)
 
     def start(self):
-        try:
-            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "50"],
-                                         stdout=self.file, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        if self.thread is not None:
+            self.thread.start()
+
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
 
     def stop(self):
-        if self.proc is None:
-            return None
-        time.sleep(0.15)
-        self.proc.terminate()
-        try:
-            self.proc.wait(5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.file.flush()
-        rows = [r.split(", ") for r in open(self.file.name).read().strip().splitlines() if r.strip()]
-        os.unlink(self.file.name)
-        sm, smax, reasons, util = [], 0.0, set(), []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            try:
-                s, mx, u = float(r[2]), float(r[3]), float(r[5])
-            except (ValueError, IndexError):
-                continue
-            smax = max(smax, mx)
-            util.append(u)
-            if u > 0:
-                sm.append(s)
-                for nm, v in zip(names, r[7:11]):
-                    if v.strip().lower() == "active":
-                        reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax or None,
-                "reasons": sorted(reasons), "samples": len(rows), "samples_busy": len(sm)}
+        if self.thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "error": self.error}
+        self.stop_ev.set()
+        self.thread.join(1.0)
+        inside = [(sm, rs) for (t, sm, rs) in self.samples if self.t0 <= t <= self.t1]
+        reasons = sorted({nm for (_, rs) in inside for bit, nm in self.REASONS.items() if rs & bit})
+        out = {"sm_mhz": statistics.median([sm for sm, _ in inside]) if inside else None,
+               "sm_max_mhz": self.smax, "reasons": reasons, "samples": len(inside), "source": "nvml, 2 ms"}
+        if inside:
+            out["sm_mhz_min"] = min(sm for sm, _ in inside)
+        if self.error:
+            out["error"] = self.error
+        return out
 
 
 def dist_setup():
@@ -216,7 +232,7 @@ def reference_arm(args, wl):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba2_2p7b")
@@ -257,17 +273,18 @@ def main():
         step()
     torch.cuda.synchronize()
 
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev)
     clocks.start()
-    time.sleep(0.2)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(ws)
     torch.cuda.synchronize()
+    clocks.mark_start()
     ev0.record(stream)
     for _ in range(args.steps):
         step()
     ev1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark_end()
     barrier(ws)
     clk = clocks.stop()
     ms = ev0.elapsed_time(ev1) / args.steps

@@ -6,14 +6,22 @@
 // stays on chip. Per block (the four steps of "SSD 算法：分块和状态传递" in the
 // Mamba-2 SSD write-up, with the block decomposition of "SSD 算法：分块矩阵分解"):
 //   step 0  A_cs[l] = sum_{j<=l} dt_j A_h            (within the block, log2 domain)
-//   step 1  G = C B^T on tensor cores (TMEM), then G'[l,s] = G[l,s] exp(A_cs[l]-A_cs[s]) dt_s
-//           for s <= l (0 above the diagonal) plus D_h on the diagonal, written back to
-//           TMEM as bf16, and Y_diag = G' X with G' as the TMEM A operand (this also
-//           yields the D x skip term)
-//   step 2  dS^T = B^T X' on tensor cores, X'[s,:] = exp(A_cs[127]-A_cs[s]) dt_s x_s
-//   step 3  S <- exp(A_cs[127]) S + dS                 (fp32, registers)
+//   step 1  G = C B^T on tensor cores (TMEM), G' = causal part of G written back to TMEM
+//           as bf16, and Y_diag = G' X'' with G' as the TMEM A operand
+//   step 2  dS^T = B^T X'' on tensor cores
+//   step 3  S <- exp(A_cs[127]) S + exp(A_cs[127] - m) dS            (fp32, registers)
 //   step 4  Y_off = C S_in^T on tensor cores (S_in in bf16 shared memory), and
-//           y = Y_diag + exp(A_cs[l]) Y_off
+//           y = exp(A_cs[l] - m) Y_diag + exp(A_cs[l]) Y_off
+// The decay exp(A_cs[l] - A_cs[s]) of the masked block is split at the block's
+// reference m (the middle of the range of A_cs): exp(A_cs[l] - m) is a row factor
+// applied in the epilogue and exp(m - A_cs[s]) dt_s a column factor applied to x,
+// X''[s,:] = exp(m - A_cs[s]) dt_s x_s, in place in shared memory. Both factors stay
+// within 2^64 when the block's A_cs range is at most 128 (log2 units), which holds for
+// any decay that leaves more than 2^-128 of a state after 128 tokens. The D skip term
+// rides on the diagonal of G' as D_h / dt_l. A block outside those bounds (a wider
+// range, or a token with |dt| < 2^-40) takes the exact form instead: G'[l,s] =
+// G[l,s] exp(A_cs[l] - A_cs[s]) dt_s (+ D_h on the diagonal) elementwise, Y_diag = G' X,
+// and m = A_cs[127], so the same steps 2-4 apply.
 // A chunk argument of 256 is evaluated as two 128-token diagonal blocks; the
 // 128x128 block between them goes through the state (its low-rank factor), which
 // is the same matrix product re-associated.
@@ -24,10 +32,10 @@
 // CTA holding the rest runs it last, so the hand-over is ready long before it is
 // read. The wait for it is bounded all the same.
 //
-// Warp roles (384 threads): warp 0 loads (TMA + dt) and issues Y_diag; warps 1, 2
+// Warp roles (384 threads): warp 0 loads (TMA + dt), runs step 0 and issues Y_diag; warps 1, 2
 // and 3 issue C B^T, the chunk states and Y_off (one issuing thread per product:
 // an MMA instruction keeps its issuing warp busy for ~100 cycles, so the products
-// are issued in parallel); warps 4-7 ("T") do step 0, G' and X'; warps 8-11 ("E")
+// are issued in parallel); warps 4-7 ("T") do X'' and G'; warps 8-11 ("E")
 // run the state chain and the epilogue. Every wait is bounded: on timeout the CTA
 // raises a status word in the workspace, drains its own TMA loads and MMAs, frees
 // TMEM and returns.
@@ -66,14 +74,12 @@ struct Cfg {
     static constexpr int kOffXp = kStages * kStageBytes;
     static constexpr int kOffSt = kOffXp + kXBytes;
     static constexpr int kOffSmall = kOffSt + kStBufs * kStBytes;
-    // per stage: dt, A_cs (log2 domain), the two column-factor arrays of step 1 and the block total
+    // per stage: dt, A_cs (log2 domain) and the block scalars {A_cs[127], m, exact?, valid tokens}
     static constexpr int kOffDts = kOffSmall;                       // float [kStages][128]
     static constexpr int kOffAcs = kOffDts + kStages * kQ * 4;      // float [kStages][128]
-    static constexpr int kOffCfE = kOffAcs + kStages * kQ * 4;      // float [kStages][128]
-    static constexpr int kOffCfS = kOffCfE + kStages * kQ * 4;      // float [kStages][128]
-    static constexpr int kOffTot = kOffCfS + kStages * kQ * 4;      // float [kStages][4]
-    static constexpr int kOffBar = kOffTot + kStages * 16;          // uint64 barriers
-    static constexpr int kNumBars = 2 * kStages + 13 + kStBufs + 2 * kYBufs;
+    static constexpr int kOffBlk = kOffAcs + kStages * kQ * 4;      // float4 [kStages]
+    static constexpr int kOffBar = kOffBlk + kStages * 16;          // uint64 barriers
+    static constexpr int kNumBars = 3 * kStages + 11 + kStBufs + 2 * kYBufs;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;         // tmem base, abort flag
     static constexpr int kSmemBytes = kOffMisc + 16;
     static constexpr int kSmemAlloc = kSmemBytes + 1024;            // slack for 1024-B alignment
@@ -304,6 +310,14 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 #undef SSD_R8
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// The same wait, with the registers of an earlier tcgen05.ld as operands, so that the
+// compiler cannot move a use of them above it (needed when other loads are in flight).
+#define SSD_W8(i) "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]), \
+                  "+r"(r[i + 6]), "+r"(r[i + 7])
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : SSD_W8(0), SSD_W8(8), SSD_W8(16), SSD_W8(24)::"memory");
+}
+#undef SSD_W8
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
@@ -324,6 +338,29 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
+// Packed fp32 pairs (sm_100): s = g s + d r on two lanes of the state at once, and
+// the epilogue's el * ys + rd * yd on two columns at once.
+__device__ __forceinline__ void fma2_state(float &s0, float &s1, float g, float d, uint32_t r0, uint32_t r1) {
+    asm("{\n\t.reg .b64 s, q, gg, dd;\n\t"
+        "mov.b64 s, {%0, %1};\n\tmov.b64 q, {%4, %5};\n\t"
+        "mov.b64 gg, {%2, %2};\n\tmov.b64 dd, {%3, %3};\n\t"
+        "mul.rn.f32x2 q, q, dd;\n\tfma.rn.f32x2 s, gg, s, q;\n\t"
+        "mov.b64 {%0, %1}, s;\n\t}"
+        : "+f"(s0), "+f"(s1)
+        : "f"(g), "f"(d), "r"(r0), "r"(r1));
+}
+__device__ __forceinline__ uint32_t epi2_bf16(float el, float rd, uint32_t ys0, uint32_t ys1, uint32_t yd0,
+                                              uint32_t yd1) {
+    uint32_t o;
+    asm("{\n\t.reg .b64 a, b, e, r;\n\t.reg .f32 lo, hi;\n\t"
+        "mov.b64 a, {%3, %4};\n\tmov.b64 b, {%5, %6};\n\t"
+        "mov.b64 e, {%1, %1};\n\tmov.b64 r, {%2, %2};\n\t"
+        "mul.rn.f32x2 b, b, r;\n\tfma.rn.f32x2 a, e, a, b;\n\t"
+        "mov.b64 {lo, hi}, a;\n\tcvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
+        : "=r"(o)
+        : "f"(el), "f"(rd), "r"(ys0), "r"(ys1), "r"(yd0), "r"(yd1));
+    return o;
+}
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
@@ -343,6 +380,35 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volati
 // block total is returned. Every warp runs the same sequence of operations, so
 // every warp gets bit-identical values.
 // ---------------------------------------------------------------------------------
+
+// Exact form of G' for one warp's 32 rows (lane quarter qtr): every element of the causal
+// part takes its own exponential, D_h on the diagonal. Out of line: it runs only for blocks
+// whose decay range is too wide for the factored form.
+__device__ __noinline__ void gprime_exact(uint32_t gaddr, int qtr, int row, float acs_r, const float *acsW,
+                                          const float *dk, float Dh) {
+#pragma unroll 1
+    for (int jb = 0; jb < 4; ++jb) {
+        uint32_t out[16];
+        if (jb > qtr) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) out[i] = 0u;
+        } else {
+            uint32_t r[32];
+            tmem_ld32(gaddr + 32 * jb, r);
+            tmem_wait_ld(r);
+#pragma unroll 4
+            for (int i = 0; i < 16; ++i) {
+                const int s = 32 * jb + 2 * i;
+                float v0 = s <= row ? __uint_as_float(r[2 * i]) * ex2(acs_r - acsW[s]) * dk[s] : 0.f;
+                float v1 = s + 1 <= row ? __uint_as_float(r[2 * i + 1]) * ex2(acs_r - acsW[s + 1]) * dk[s + 1] : 0.f;
+                v0 += s == row ? Dh : 0.f;
+                v1 += s + 1 == row ? Dh : 0.f;
+                out[i] = pack_bf16(v0, v1);
+            }
+        }
+        tmem_st16(gaddr + 16 * jb, out);
+    }
+}
 
 // Bounded spin on a hand-over counter in global memory.
 __device__ __noinline__ bool wait_flag(const int *flag, int want, volatile int *abort_flag, int *status) {
@@ -373,16 +439,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     float *dts = reinterpret_cast<float *>(sm + Cf::kOffDts);
     float *acs_s = reinterpret_cast<float *>(sm + Cf::kOffAcs);
-    float *cfe_s = reinterpret_cast<float *>(sm + Cf::kOffCfE);
-    float *cfs_s = reinterpret_cast<float *>(sm + Cf::kOffCfS);
-    float *tot_s = reinterpret_cast<float *>(sm + Cf::kOffTot);
+    float4 *blk_s = reinterpret_cast<float4 *>(sm + Cf::kOffBlk);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + Cf::kOffBar);
     uint64_t *full = bar;                // [S]   stage loaded (TMA bytes + dt)
     uint64_t *empty = full + S;          // [S]   stage consumed: 4 issuer commits + 4 T warps + 4 E warps
     uint64_t *gfull = empty + S;         // [2]   C B^T in score buffer j
-    uint64_t *gp = gfull + 2;            // [2]   G' written back to score buffer j (T)
-    uint64_t *xpr = gp + 2;              // [1]   X' written (T)
-    uint64_t *dsdone = xpr + 1;          // [2]   chunk state of block t done, buffer t % 2
+    uint64_t *gp = gfull + 2;            // [2]   G' written back to score buffer j, and X'' (T)
+    uint64_t *xpr = gp + 2;              // [S]   X'' of stage k written (T)
+    uint64_t *dsdone = xpr + S;          // [2]   chunk state of block t done, buffer t % 2
     uint64_t *dsfree = dsdone + 2;       // [2]   chunk state of block t read by E
     uint64_t *ydd = dsfree + 2;          // [2]   Y_diag of block t done (score buffer t % 2 reusable)
     uint64_t *sready = ydd + 2;          // [SB]  S_in^T of block t written (E)
@@ -411,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&dsfree[i], 128);
             mbar_init(&ydd[i], 1);
         }
-        mbar_init(xpr, 128);
+        for (int i = 0; i < S; ++i) mbar_init(&xpr[i], 128);
         for (int i = 0; i < SB; ++i) mbar_init(&sready[i], 128);
         for (int i = 0; i < YB; ++i) {
             mbar_init(&yfull[i], 2);
@@ -445,46 +509,62 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kIdY = idesc(128, 64, false, true);
 
     if (warp == kWarpTma) {
-        // ------------------------------------------------------------- loads + Y_diag issue
+        // ------------------------------------------------------------- loads, step 0, Y_diag issue
         // Task t's stage is loaded, then Y_diag of task t-1 is issued (with one stage, Y_diag of
-        // t-1 goes first: the stage of t is released only once Y_diag of t-1 is done).
-        float dtn[4], acn[4], cen[4], csn[4], totn = 0.f;
+        // t-1 goes first: the stage of t is released only once Y_diag of t-1 is done), then step 0
+        // of task t+1 runs on dt that was fetched one task earlier, and dt of task t+2 is fetched.
         const uint64_t pol_keep = policy_evict_last(), pol_stream = policy_evict_first();
-        // dt of the next task, fetched into registers one task ahead, and its step 0: the
-        // within-block cumsum of dt * A_h (log2 domain) and the column factors of step 1,
-        // cfE[s] = exp(A_end - A_s) dt_s and cfS[s] = exp(A_start - A_s) dt_s, referenced to
-        // the last and the first entry of the 32-entry sub-block of s.
+        // Lane i handles tokens 4 i .. 4 i + 3 of a block.
+        float raw[4], a_raw = 0.f;  // dt and A_h of the task after the prepared one
+        int nvalid_raw = 0;
+        float4 dtn, acn;            // prepared step 0 of the next task to load
+        float4 blkn = make_float4(0.f, 0.f, 0.f, 0.f);
         auto fetch = [&](int t) {
             const long long gi = sh.task(t);
             const int sidx = (int)(gi / nc), c = (int)(gi % nc), b = sidx / H, h = sidx % H;
-            const float a2 = __ldg(prm.A + h) * kLog2e;
-            float carry = 0.f;
+            a_raw = __ldg(prm.A + h);
+            nvalid_raw = (int)min((long long)kQ, L - (long long)c * kQ);
+            const long long t0 = (long long)c * kQ + 4 * lane;
+            const __nv_bfloat16 *src = prm.dt + ((long long)b * L + t0) * H + h;
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const long long tt = (long long)c * kQ + lane + 32 * m;
-                dtn[m] = tt < L ? __bfloat162float(prm.dt[((long long)b * L + tt) * H + h]) : 0.f;
-                float x = dtn[m] * a2;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float u = __shfl_up_sync(0xffffffffu, x, o);
-                    if (lane >= o) x += u;
-                }
-                x += carry;
-                acn[m] = x;
-                carry = __shfl_sync(0xffffffffu, x, 31);
-                const float vbeg = __shfl_sync(0xffffffffu, x, 0);
-                cen[m] = ex2(carry - x) * dtn[m];
-                csn[m] = ex2(vbeg - x) * dtn[m];
-            }
-            totn = carry;
+            for (int m = 0; m < 4; ++m) raw[m] = t0 + m < L ? __bfloat162float(src[(long long)m * H]) : 0.f;
         };
-        auto issue_yd = [&](int t) -> bool {  // Y_diag = G' X with G' in TMEM   (M = l, N = p, K = s)
+        // Step 0 on the fetched dt: the within-block cumsum of dt * A_h (log2 domain), its
+        // range, the reference m in the middle of it, and whether the factored form is safe.
+        auto prep = [&]() {
+            const float a2 = a_raw * kLog2e;
+            dtn = make_float4(raw[0], raw[1], raw[2], raw[3]);
+            const float v0 = dtn.x * a2, v1 = fmaf(dtn.y, a2, v0), v2 = fmaf(dtn.z, a2, v1), v3 = fmaf(dtn.w, a2, v2);
+            float incl = v3;  // inclusive scan of the lanes' sums
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float u = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += u;
+            }
+            const float excl = incl - v3;
+            acn = make_float4(excl + v0, excl + v1, excl + v2, incl);
+            const float tot = __shfl_sync(0xffffffffu, incl, 31);
+            float mx = fmaxf(fmaxf(acn.x, acn.y), fmaxf(acn.z, acn.w));
+            float mn = fminf(fminf(acn.x, acn.y), fminf(acn.z, acn.w));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            }
+            const int nv = nvalid_raw - 4 * lane;  // valid tokens of this lane: min(max(nv, 0), 4)
+            const bool dt_ok = (nv <= 0 || fabsf(dtn.x) >= 0x1p-40f) && (nv <= 1 || fabsf(dtn.y) >= 0x1p-40f) &&
+                               (nv <= 2 || fabsf(dtn.z) >= 0x1p-40f) && (nv <= 3 || fabsf(dtn.w) >= 0x1p-40f);
+            // (mx - mn <= 128 is false for NaN, which then takes the exact form)
+            const bool factored = __all_sync(0xffffffffu, dt_ok) && (mx - mn <= 128.f);
+            blkn = make_float4(tot, factored ? 0.5f * (mx + mn) : tot, factored ? 0.f : 1.f, (float)nvalid_raw);
+        };
+        auto issue_yd = [&](int t) -> bool {  // Y_diag = G' X'' with G' in TMEM   (M = l, N = p, K = s)
             const int k = t % S, j = t & 1, yb = t % YB;
             if (!wait_warp(&gp[j], (uint32_t)(t >> 1) & 1u, abort_flag, status)) return false;
             if (t >= YB && !wait_warp(&yfree[yb], (uint32_t)((t - YB) / YB) & 1u, abort_flag, status)) return false;
             if (lane == 0) {
                 tc_fence_after();
-                const uint32_t xa = smem_u32(stage_x(k));
+                const uint32_t xa = smem_u32(stage_x(k));  // X'' in place (x itself in the exact form)
 #pragma unroll
                 for (int kk = 0; kk < kQ / 16; ++kk)
                     mma_ts(tmem + Cf::kTmY + 128 * yb, tmem + 128 * j + 8 * kk, sdesc(xa + kk * 2048, 1024, 1024),
@@ -496,26 +576,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             return true;
         };
-        if (ntask > 0) fetch(0);
-        int nl = 0, nyd = 0;
+        if (ntask > 0) {
+            fetch(0);
+            prep();
+            if (ntask > 1) fetch(1);
+        }
+        int nl = 0;
         bool ok = true;
         for (int t = 0; ok && t < ntask; ++t) {
             const int k = t % S;
-            if (S == 1 && t >= 1) {
-                if (!(ok = issue_yd(t - 1))) break;
-                nyd = t;
-            }
+            if (S == 1 && t >= 1 && !(ok = issue_yd(t - 1))) break;
             if (t >= S && !(ok = wait_warp(&empty[k], (uint32_t)((t / S) - 1) & 1u, abort_flag, status))) break;
             const long long gi = sh.task(t);
             const int sidx = (int)(gi / nc), c = (int)(gi % nc), b = sidx / H, h = sidx % H;
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                dts[k * kQ + lane + 32 * m] = dtn[m];
-                acs_s[k * kQ + lane + 32 * m] = acn[m];
-                cfe_s[k * kQ + lane + 32 * m] = cen[m];
-                cfs_s[k * kQ + lane + 32 * m] = csn[m];
-            }
-            if (lane == 0) tot_s[k * 4] = totn;
+            reinterpret_cast<float4 *>(dts + k * kQ)[lane] = dtn;
+            reinterpret_cast<float4 *>(acs_s + k * kQ)[lane] = acn;
+            if (lane == 0) blk_s[k] = blkn;
             __syncwarp();
             if (lane == 0) {
                 const int t0 = c * kQ, g = h / hpg;
@@ -528,13 +604,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
             nl = t + 1;
-            if (t + 1 < ntask) fetch(t + 1);
-            if (S > 1 && t >= 1) {
-                if (!(ok = issue_yd(t - 1))) break;
-                nyd = t;
+            if (S > 1 && t >= 1 && !(ok = issue_yd(t - 1))) break;
+            if (t + 1 < ntask) {
+                prep();
+                if (t + 2 < ntask) fetch(t + 2);
             }
         }
-        if (ok && ntask > 0 && issue_yd(ntask - 1)) nyd = ntask;
+        if (ok && ntask > 0) issue_yd(ntask - 1);
         if (lane == 0) mma_commit(fin);
         // drain: loads still in flight land before the CTA exits
         if (lane == 0) {
@@ -570,18 +646,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else if (warp == kWarpDs) {
-        // ------------------------------------------------------------- dS^T = B^T X'   (M = n, N = p, K = s)
+        // ------------------------------------------------------------- dS^T = B^T X''   (M = n, N = p, K = s)
         if (lane == 0) {
             for (int t = 0; t < ntask; ++t) {
                 const int k = t % S, j = t & 1;
-                if (!wait_phase(xpr, (uint32_t)t & 1u, abort_flag, status)) break;
+                if (!wait_phase(&xpr[k], (uint32_t)(t / S) & 1u, abort_flag, status)) break;
                 if (Cf::kDsInG) {  // T is done reading C B^T from the half this state goes to
                     if (!wait_phase(&gp[j], (uint32_t)(t >> 1) & 1u, abort_flag, status)) break;
                 } else if (t >= 1) {
                     if (!wait_phase(&dsfree[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u, abort_flag, status)) break;
                 }
                 tc_fence_after();
-                const uint32_t ba = smem_u32(stage_b(k)), xa = smem_u32(xp);
+                // X'' in place in the stage, or (exact form) X' in its own buffer
+                const bool exact = blk_s[k].z != 0.f;
+                const uint32_t ba = smem_u32(stage_b(k)), xa = smem_u32(exact ? xp : stage_x(k));
 #pragma unroll
                 for (int hf = 0; hf < N / 128; ++hf) {
 #pragma unroll
@@ -619,10 +697,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else if (warp < kWarpE) {
-        // ------------------------------------------------------------- T: step 0, G', X'
+        // ------------------------------------------------------------- T: X'' and G'
         const int qtr = warp & 3;  // TMEM lane quarter of this warp: rows 32 qtr .. 32 qtr + 31
         const int row = (qtr << 5) | lane;
         const uint32_t lane_off = (uint32_t)(qtr * 32) << 16;
+        // Row `row` of x (64 bf16, 128-byte swizzled) scaled by w, from src to dst.
+        auto scale_row = [&](const unsigned char *src, unsigned char *dst, float w) {
+#pragma unroll 1
+            for (int ch = 0; ch < 8; ++ch) {
+                const uint4 xv = *reinterpret_cast<const uint4 *>(src + swz(row, ch));
+                uint4 o;
+                o.x = pack_bf16(w * bf16_lo(xv.x), w * bf16_hi(xv.x));
+                o.y = pack_bf16(w * bf16_lo(xv.y), w * bf16_hi(xv.y));
+                o.z = pack_bf16(w * bf16_lo(xv.z), w * bf16_hi(xv.z));
+                o.w = pack_bf16(w * bf16_lo(xv.w), w * bf16_hi(xv.w));
+                *reinterpret_cast<uint4 *>(dst + swz(row, ch)) = o;
+            }
+        };
         for (int t = 0; t < ntask; ++t) {
             const int k = t % S, j = t & 1;
             const int h = (int)((sh.task(t) / nc) % H);
@@ -630,90 +721,61 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!wait_warp(&full[k], (uint32_t)(t / S) & 1u, abort_flag, status)) break;
             const float *dk = dts + k * kQ;
             const float *acsW = acs_s + k * kQ;
-            const float *cfE = cfe_s + k * kQ;
-            const float *cfS = cfs_s + k * kQ;
-            const float tot = tot_s[k * 4];
-            const float acs_r = acsW[row];
-            const float acs_q0 = acsW[32 * qtr];
-            const float span_q = acs_q0 - acsW[32 * qtr + 31];
-            // G' = (C B^T) o decay o dt (+ D on the diagonal), in place in TMEM as packed bf16 pairs
+            const float4 blk = blk_s[k];  // {A_cs[127], m, exact?, valid tokens}
+            const bool exact = blk.z != 0.f;  // warp-uniform
+            const float acs_r = acsW[row], dt_r = dk[row];
+            const uint32_t gaddr = tmem + 128 * j + lane_off;
+            // X''[row,:] = exp(m - A_cs[row]) dt_row x_row, in place; in the exact form (m = A_cs[127])
+            // into its own buffer, once the previous chunk-state MMA is done reading that
+            if (exact && t > 0 &&
+                !wait_warp(&dsdone[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u, abort_flag, status))
+                break;
+            scale_row(stage_x(k), exact ? xp : stage_x(k), ex2(blk.y - acs_r) * dt_r);
+            fence_proxy_async();
+            mbar_arrive(&xpr[k]);
             if (!wait_warp(&gfull[j], (uint32_t)(t >> 1) & 1u, abort_flag, status)) break;
             tc_fence_after();
-            {
-                const uint32_t gaddr = tmem + 128 * j + lane_off;
-                // factors of the diagonal sub-block stay inside fp32 range when its decay span is
-                // below 2^120; otherwise every element takes its own exponential
-                const bool diag_factored = span_q < 120.f;  // warp-uniform
-                const float rf_diag = ex2(acs_r - acs_q0);
+            if (!exact) {
+                const float dinv = dt_r != 0.f ? Dh / dt_r : 0.f;  // dt = 0 only on padding rows here
+                // 32-column blocks jb < qtr lie below the diagonal: plain conversion to bf16 pairs
 #pragma unroll 1
-                for (int jb = 0; jb < 4; ++jb) {
-                    uint32_t out[16];
-                    if (jb > qtr) {
+                for (int jb = 0; jb < qtr; ++jb) {
+                    uint32_t r[32], out[16];
+                    tmem_ld32(gaddr + 32 * jb, r);
+                    tmem_wait_ld(r);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) out[i] = 0u;
-                    } else {
-                        uint32_t r[32];
-                        tmem_ld32(gaddr + 32 * jb, r);
-                        tmem_wait_ld();
-                        if (jb < qtr) {
-                            const float rf = ex2(acs_r - acsW[32 * jb + 31]);
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const float2 cf = *reinterpret_cast<const float2 *>(cfE + 32 * jb + 2 * i);
-                                out[i] = pack_bf16(__uint_as_float(r[2 * i]) * rf * cf.x,
-                                                   __uint_as_float(r[2 * i + 1]) * rf * cf.y);
-                            }
-                        } else if (diag_factored) {
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const int s = 32 * jb + 2 * i;
-                                const float2 cf = *reinterpret_cast<const float2 *>(cfS + s);
-                                float v0 = s <= row ? __uint_as_float(r[2 * i]) * rf_diag * cf.x : 0.f;
-                                float v1 = s + 1 <= row ? __uint_as_float(r[2 * i + 1]) * rf_diag * cf.y : 0.f;
-                                v0 += s == row ? Dh : 0.f;
-                                v1 += s + 1 == row ? Dh : 0.f;
-                                out[i] = pack_bf16(v0, v1);
-                            }
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const int s = 32 * jb + 2 * i;
-                                float v0 = s <= row ? __uint_as_float(r[2 * i]) * ex2(acs_r - acsW[s]) * dk[s] : 0.f;
-                                float v1 =
-                                    s + 1 <= row ? __uint_as_float(r[2 * i + 1]) * ex2(acs_r - acsW[s + 1]) * dk[s + 1]
-                                                 : 0.f;
-                                v0 += s == row ? Dh : 0.f;
-                                v1 += s + 1 == row ? Dh : 0.f;
-                                out[i] = pack_bf16(v0, v1);
-                            }
-                        }
-                    }
+                    for (int i = 0; i < 16; ++i)
+                        out[i] = pack_bf16(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
                     tmem_st16(gaddr + 16 * jb, out);
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&gp[j]);
-            }
-            // X' (the previous task's chunk-state MMA must be done reading X')
-            if (t > 0 && !wait_warp(&dsdone[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u, abort_flag, status)) break;
-            {
-                const float w = ex2(tot - acs_r) * dk[row];
-                const unsigned char *xs = stage_x(k);
+                {  // block qtr holds the diagonal: mask s > row, D_h / dt_l on s == row
+                    uint32_t r[32], out[16];
+                    tmem_ld32(gaddr + 32 * qtr, r);
+                    tmem_wait_ld(r);
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const uint4 xv = *reinterpret_cast<const uint4 *>(xs + swz(row, ch));
-                    uint4 o;
-                    o.x = pack_bf16(w * bf16_lo(xv.x), w * bf16_hi(xv.x));
-                    o.y = pack_bf16(w * bf16_lo(xv.y), w * bf16_hi(xv.y));
-                    o.z = pack_bf16(w * bf16_lo(xv.z), w * bf16_hi(xv.z));
-                    o.w = pack_bf16(w * bf16_lo(xv.w), w * bf16_hi(xv.w));
-                    *reinterpret_cast<uint4 *>(xp + swz(row, ch)) = o;
+                    for (int i = 0; i < 16; ++i) {
+                        const int s = 2 * i, rl = lane;  // offsets within the block
+                        float v0 = s <= rl ? __uint_as_float(r[2 * i]) : 0.f;
+                        float v1 = s + 1 <= rl ? __uint_as_float(r[2 * i + 1]) : 0.f;
+                        v0 += s == rl ? dinv : 0.f;
+                        v1 += s + 1 == rl ? dinv : 0.f;
+                        out[i] = pack_bf16(v0, v1);
+                    }
+                    tmem_st16(gaddr + 16 * qtr, out);
                 }
-                fence_proxy_async();
-                mbar_arrive(xpr);
+                uint32_t zero[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) zero[i] = 0u;
+#pragma unroll 1
+                for (int jb = qtr + 1; jb < 4; ++jb) tmem_st16(gaddr + 16 * jb, zero);
+            } else {
+                gprime_exact(gaddr, qtr, row, acs_r, acsW, dk, Dh);
             }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&gp[j]);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[k]);  // this warp is done with X and dt of the stage
+            if (lane == 0) mbar_arrive(&empty[k]);  // this warp is done with the stage
         }
     } else {
         // ------------------------------------------------------------- E: state chain + epilogue
@@ -798,25 +860,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const long long gi = sh.task(t);
             const int h = (int)((gi / nc) % H), c = (int)(gi % nc);
             if (!(ok = wait_warp(&full[k], (uint32_t)(t / S) & 1u, abort_flag, status))) break;
-            const float tot = tot_s[k * 4];
+            const float4 blk = blk_s[k];  // {A_cs[127], m, exact?, valid tokens}
             const float acs_r = acs_s[k * kQ + row];
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[k]);  // done with the step-0 values of the stage
-            // step 3: S <- exp(A_cs[end]) S + dS
+            // step 3: S <- exp(A_cs[127]) S + exp(A_cs[127] - m) dS
             if (!(ok = wait_warp(&dsdone[j], (uint32_t)(t >> 1) & 1u, abort_flag, status))) break;
             tc_fence_after();
             {
-                const float gam = ex2(tot);
+                const float gam = ex2(blk.x), dsc = ex2(blk.x - blk.y);
 #pragma unroll
                 for (int i = 0; i < NH; ++i) {
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         uint32_t r[32];
                         tmem_ld32(tmem + ds_col(t) + 64 * i + 32 * half + lane_off, r);
-                        tmem_wait_ld();
+                        tmem_wait_ld(r);
 #pragma unroll
-                        for (int q = 0; q < 32; ++q)
-                            Sr[i][32 * half + q] = fmaf(gam, Sr[i][32 * half + q], __uint_as_float(r[q]));
+                        for (int q = 0; q < 32; q += 2)
+                            fma2_state(Sr[i][32 * half + q], Sr[i][32 * half + q + 1], gam, dsc, r[q], r[q + 1]);
                     }
                 }
                 tc_fence_before();
@@ -830,17 +892,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (last_of_piece && !(ok = load_init(t + 1))) break;
                 write_st(t + 1);
             }
-            // epilogue: y = Y_diag + exp(A_cs[l]) Y_off   (D x is inside Y_diag)
+            // epilogue: y = exp(A_cs[l] - m) Y_diag + exp(A_cs[l]) Y_off   (D x is inside Y_diag;
+            // the exact form has no row factor)
             if (!(ok = wait_warp(&yfull[yb], (uint32_t)(t / YB) & 1u, abort_flag, status))) break;
             tc_fence_after();
             {
                 // y rows of this warp (32 tokens x 64 values) are staged, 128-byte swizzled, in its
                 // 4 KB slice of the S^T buffer of task t (free: Y_off of task t is done) and written
                 // by one bulk tensor store.
-                const float el = ex2(acs_r);
+                const float el = ex2(acs_r), rd = blk.z != 0.f ? 1.f : ex2(acs_r - blk.y);
                 unsigned char *stage_y = st_buf(t % SB);
                 const uint32_t ya = tmem + Cf::kTmY + 128 * yb + lane_off;
-#pragma unroll
+#pragma unroll 1
                 for (int qq = 0; qq < 4; ++qq) {  // 16 columns at a time
                     uint32_t yd[16], ys[16];
                     tmem_ld16(ya + 16 * qq, yd);
@@ -852,9 +915,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     uint32_t o[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        o[e] = pack_bf16(fmaf(el, __uint_as_float(ys[2 * e]), __uint_as_float(yd[2 * e])),
-                                         fmaf(el, __uint_as_float(ys[2 * e + 1]), __uint_as_float(yd[2 * e + 1])));
+                    for (int e = 0; e < 8; ++e) o[e] = epi2_bf16(el, rd, ys[2 * e], ys[2 * e + 1], yd[2 * e], yd[2 * e + 1]);
                     *reinterpret_cast<uint4 *>(stage_y + swz(row, 2 * qq)) = make_uint4(o[0], o[1], o[2], o[3]);
                     *reinterpret_cast<uint4 *>(stage_y + swz(row, 2 * qq + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
                 }
