@@ -78,7 +78,8 @@ struct Cfg {
     static constexpr int kOffDts = kOffSmall;                       // float [kStages][128]
     static constexpr int kOffAcs = kOffDts + kStages * kQ * 4;      // float [kStages][128]
     static constexpr int kOffBlk = kOffAcs + kStages * kQ * 4;      // float4 [kStages]
-    static constexpr int kOffBar = kOffBlk + kStages * 16;          // uint64 barriers
+    static constexpr int kOffCrd = kOffBlk + kStages * 16;          // int4 [kStages]: b, h, c, last-of-piece
+    static constexpr int kOffBar = kOffCrd + kStages * 16;          // uint64 barriers
     static constexpr int kNumBars = 3 * kStages + 11 + kStBufs + 2 * kYBufs;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;         // tmem base, abort flag
     static constexpr int kSmemBytes = kOffMisc + 16;
@@ -440,6 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *dts = reinterpret_cast<float *>(sm + Cf::kOffDts);
     float *acs_s = reinterpret_cast<float *>(sm + Cf::kOffAcs);
     float4 *blk_s = reinterpret_cast<float4 *>(sm + Cf::kOffBlk);
+    int4 *crd_s = reinterpret_cast<int4 *>(sm + Cf::kOffCrd);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + Cf::kOffBar);
     uint64_t *full = bar;                // [S]   stage loaded (TMA bytes + dt)
     uint64_t *empty = full + S;          // [S]   stage consumed: 4 issuer commits + 4 T warps + 4 E warps
@@ -519,9 +521,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         int nvalid_raw = 0;
         float4 dtn, acn;            // prepared step 0 of the next task to load
         float4 blkn = make_float4(0.f, 0.f, 0.f, 0.f);
+        int4 crd_raw = make_int4(0, 0, 0, 0), crd_n = crd_raw;  // {b, h, c, last of its piece}
+        // Task coordinates advance by one block at a time except where the share's order
+        // jumps (at most twice), so the divisions run only there.
+        long long cur_gi = -2;
+        int cur_c = 0, cur_b = 0, cur_h = 0;
         auto fetch = [&](int t) {
             const long long gi = sh.task(t);
-            const int sidx = (int)(gi / nc), c = (int)(gi % nc), b = sidx / H, h = sidx % H;
+            if (gi == cur_gi + 1 && cur_c + 1 < nc) {
+                ++cur_c;
+            } else if (gi == cur_gi + 1) {
+                cur_c = 0;
+                if (++cur_h == H) {
+                    cur_h = 0;
+                    ++cur_b;
+                }
+            } else {
+                const int sidx = (int)(gi / nc);
+                cur_c = (int)(gi - (long long)sidx * nc);
+                cur_b = sidx / H;
+                cur_h = sidx - cur_b * H;
+            }
+            cur_gi = gi;
+            const int b = cur_b, h = cur_h, c = cur_c;
+            crd_raw = make_int4(b, h, c, (c == nc - 1 || gi == sh.hi - 1) ? 1 : 0);
             a_raw = __ldg(prm.A + h);
             nvalid_raw = (int)min((long long)kQ, L - (long long)c * kQ);
             const long long t0 = (long long)c * kQ + 4 * lane;
@@ -533,6 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // range, the reference m in the middle of it, and whether the factored form is safe.
         auto prep = [&]() {
             const float a2 = a_raw * kLog2e;
+            crd_n = crd_raw;
             dtn = make_float4(raw[0], raw[1], raw[2], raw[3]);
             const float v0 = dtn.x * a2, v1 = fmaf(dtn.y, a2, v0), v2 = fmaf(dtn.z, a2, v1), v3 = fmaf(dtn.w, a2, v2);
             float incl = v3;  // inclusive scan of the lanes' sums
@@ -565,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) {
                 tc_fence_after();
                 const uint32_t xa = smem_u32(stage_x(k));  // X'' in place (x itself in the exact form)
-#pragma unroll
+#pragma unroll 1
                 for (int kk = 0; kk < kQ / 16; ++kk)
                     mma_ts(tmem + Cf::kTmY + 128 * yb, tmem + 128 * j + 8 * kk, sdesc(xa + kk * 2048, 1024, 1024),
                            kIdY, kk > 0);
@@ -587,11 +611,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int k = t % S;
             if (S == 1 && t >= 1 && !(ok = issue_yd(t - 1))) break;
             if (t >= S && !(ok = wait_warp(&empty[k], (uint32_t)((t / S) - 1) & 1u, abort_flag, status))) break;
-            const long long gi = sh.task(t);
-            const int sidx = (int)(gi / nc), c = (int)(gi % nc), b = sidx / H, h = sidx % H;
+            const int b = crd_n.x, h = crd_n.y, c = crd_n.z;
             reinterpret_cast<float4 *>(dts + k * kQ)[lane] = dtn;
             reinterpret_cast<float4 *>(acs_s + k * kQ)[lane] = acn;
-            if (lane == 0) blk_s[k] = blkn;
+            if (lane == 0) {
+                blk_s[k] = blkn;
+                crd_s[k] = crd_n;
+            }
             __syncwarp();
             if (lane == 0) {
                 const int t0 = c * kQ, g = h / hpg;
@@ -634,7 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t ca = smem_u32(stage_c(k)), ba = smem_u32(stage_b(k));
-#pragma unroll
+#pragma unroll 1
                 for (int kk = 0; kk < N / 16; ++kk) {
                     const uint32_t off = (uint32_t)((kk >> 2) * Cf::kPanelBytes + (kk & 3) * 32);
                     mma_ss(tmem + 128 * j, sdesc(ca + off, 16, 1024), sdesc(ba + off, 16, 1024), kIdG, kk > 0);
@@ -660,9 +686,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // X'' in place in the stage, or (exact form) X' in its own buffer
                 const bool exact = blk_s[k].z != 0.f;
                 const uint32_t ba = smem_u32(stage_b(k)), xa = smem_u32(exact ? xp : stage_x(k));
-#pragma unroll
+#pragma unroll 1
                 for (int hf = 0; hf < N / 128; ++hf) {
-#pragma unroll
+#pragma unroll 1
                     for (int kk = 0; kk < kQ / 16; ++kk)
                         mma_ss(tmem + ds_col(t) + 64 * hf,
                                sdesc(ba + 2 * hf * Cf::kPanelBytes + kk * 2048, Cf::kPanelBytes, 1024),
@@ -684,7 +710,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (t >= YB && !wait_phase(&yfree[yb], (uint32_t)((t - YB) / YB) & 1u, abort_flag, status)) break;
                 tc_fence_after();
                 const uint32_t ca = smem_u32(stage_c(k)), sa = smem_u32(st_buf(t % SB));
-#pragma unroll
+#pragma unroll 1
                 for (int kk = 0; kk < N / 16; ++kk) {
                     const uint32_t off = (uint32_t)((kk >> 2) * Cf::kPanelBytes + (kk & 3) * 32);
                     mma_ss(tmem + Cf::kTmY + 128 * yb + 64, sdesc(ca + off, 16, 1024), sdesc(sa + kk * 2048, 1024, 1024),
@@ -716,9 +742,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         for (int t = 0; t < ntask; ++t) {
             const int k = t % S, j = t & 1;
-            const int h = (int)((sh.task(t) / nc) % H);
-            const float Dh = prm.D ? __ldg(prm.D + h) : 0.f;
             if (!wait_warp(&full[k], (uint32_t)(t / S) & 1u, abort_flag, status)) break;
+            const float Dh = prm.D ? __ldg(prm.D + crd_s[k].y) : 0.f;
             const float *dk = dts + k * kQ;
             const float *acsW = acs_s + k * kQ;
             const float4 blk = blk_s[k];  // {A_cs[127], m, exact?, valid tokens}
@@ -849,17 +874,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 atomicAdd(prm.flags + blockIdx.x, 1);
             }
         };
-        auto piece_end = [&](int t) {  // task t is the last of its piece in this CTA's order
-            const long long gi = sh.task(t);
-            return (int)(gi % nc) == nc - 1 || gi == sh.hi - 1;
-        };
         bool ok = ntask > 0 && load_init(0);
         if (ok) write_st(0);
         for (int t = 0; ok && t < ntask; ++t) {
             const int k = t % S, j = t & 1, yb = t % YB;
-            const long long gi = sh.task(t);
-            const int h = (int)((gi / nc) % H), c = (int)(gi % nc);
             if (!(ok = wait_warp(&full[k], (uint32_t)(t / S) & 1u, abort_flag, status))) break;
+            const int4 crd = crd_s[k];  // {b, h, c, last of its piece}
+            const int h = crd.y, c = crd.z;
             const float4 blk = blk_s[k];  // {A_cs[127], m, exact?, valid tokens}
             const float acs_r = acs_s[k * kQ + row];
             __syncwarp();
@@ -884,7 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 mbar_arrive(&dsfree[j]);
             }
-            const bool last_of_piece = piece_end(t);
+            const bool last_of_piece = crd.w != 0;
             if (last_of_piece) store_final(t);
             // S_in^T of the next task. With two buffers the one it goes to was last read by
             // Y_off of task t-1, which is done (the epilogue of t-1 waited for it).
@@ -923,7 +944,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 const int r0 = c * kQ + 32 * qtr;
                 if (lane == 0 && r0 < L) {
-                    const int b = (int)(gi / nc) / H;
+                    const int b = crd.x;
                     tma_store_4d(&tm_y, stage_y + 32 * qtr * 128, 0, h, r0, b, policy_evict_first());
                     bulk_commit();
                 }
