@@ -6,25 +6,26 @@
 // stays on chip. Per block (the four steps of "SSD 算法：分块和状态传递" in the
 // Mamba-2 SSD write-up, with the block decomposition of "SSD 算法：分块矩阵分解"):
 //   step 0  A_cs[l] = sum_{j<=l} dt_j A_h            (within the block, log2 domain)
-//   step 1  G = C B^T on tensor cores (TMEM), G' = causal part of G written back to TMEM
-//           as bf16, and Y_diag = G' X'' with G' as the TMEM A operand
+//   step 1  G = C B^T on tensor cores (TMEM); G' = causal part of G written back to TMEM
+//           as bf16
 //   step 2  dS^T = B^T X'' on tensor cores
 //   step 3  S <- exp(A_cs[127]) S + exp(A_cs[127] - m) dS            (fp32, registers)
-//   step 4  Y_off = C S_in^T on tensor cores (S_in in bf16 shared memory), and
-//           y = exp(A_cs[l] - m) Y_diag + exp(A_cs[l]) Y_off
+//   step 4  Y = C (exp(m) S_in)^T + G' X'' in one TMEM accumulator (S_in in bf16 shared
+//           memory, G' as the TMEM A operand), and y = exp(A_cs[l] - m) Y
 // The decay exp(A_cs[l] - A_cs[s]) of the masked block is split at the block's
 // reference m (the middle of the range of A_cs): exp(A_cs[l] - m) is a row factor
 // applied in the epilogue and exp(m - A_cs[s]) dt_s a column factor applied to x,
-// X''[s,:] = exp(m - A_cs[s]) dt_s x_s, in place in shared memory. Both factors stay
-// within 2^64 when the block's A_cs range is at most 128 (log2 units), which holds for
-// any decay that leaves more than 2^-128 of a state after 128 tokens. The D skip term
-// rides on the diagonal of G' as D_h / dt_l. A block outside those bounds (a wider
+// X''[s,:] = exp(m - A_cs[s]) dt_s x_s, in place in shared memory; the state term
+// exp(A_cs[l]) C S_in^T shares the row factor once S_in is scaled by exp(m). All factors
+// stay within 2^64 when the block's A_cs range is at most 128 (log2 units), which holds
+// for any decay that leaves more than 2^-128 of a state after 128 tokens. The D skip
+// term rides on the diagonal of G' as D_h / dt_l. A block outside those bounds (a wider
 // range, or a token with |dt| < 2^-40) takes the exact form instead: G'[l,s] =
-// G[l,s] exp(A_cs[l] - A_cs[s]) dt_s (+ D_h on the diagonal) elementwise, Y_diag = G' X,
-// and m = A_cs[127], so the same steps 2-4 apply.
-// A chunk argument of 256 is evaluated as two 128-token diagonal blocks; the
-// 128x128 block between them goes through the state (its low-rank factor), which
-// is the same matrix product re-associated.
+// G[l,s] exp(A_cs[l] - A_cs[s]) dt_s (+ D_h on the diagonal) elementwise against x itself,
+// the rows of C scaled by exp(A_cs[l]) in place, S_in unscaled, m = A_cs[127] and y = Y.
+// A chunk argument of 256 is evaluated as two 128-token diagonal blocks; the 128x128
+// block between them goes through the state (its low-rank factor), which is the same
+// matrix product re-associated.
 //
 // A stream whose blocks fall into two CTAs' shares is cut: the CTA holding its
 // first part runs that part first and hands the state over through global memory
@@ -32,13 +33,14 @@
 // CTA holding the rest runs it last, so the hand-over is ready long before it is
 // read. The wait for it is bounded all the same.
 //
-// Warp roles (384 threads): warp 0 loads (TMA + dt), runs step 0 and issues Y_diag; warps 1, 2
-// and 3 issue C B^T, the chunk states and Y_off (one issuing thread per product:
-// an MMA instruction keeps its issuing warp busy for ~100 cycles, so the products
-// are issued in parallel); warps 4-7 ("T") do X'' and G'; warps 8-11 ("E")
-// run the state chain and the epilogue. Every wait is bounded: on timeout the CTA
-// raises a status word in the workspace, drains its own TMA loads and MMAs, frees
-// TMEM and returns.
+// Warp roles (384 threads): warp 0 loads (TMA + dt) and runs step 0; warps 1, 2 and 3
+// issue C B^T, the chunk states and Y (one issuing thread per product: an MMA
+// instruction keeps its issuing warp busy for ~100 cycles, so the products are issued
+// in parallel); warps 4-7 ("T") do X'' and G'; warps 8-11 ("E") run the state chain and
+// the epilogue. B and C, and x with its step-0 values, have separate stage barriers, so
+// the next block's B and C load as soon as the products that read them are done. Every
+// wait is bounded: on timeout the CTA raises a status word in the workspace, drains its
+// own TMA loads and MMAs, frees TMEM and returns.
 #include <cuda.h>
 
 #include <algorithm>
@@ -57,14 +59,12 @@ constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
 
 template <int N>
 struct Cfg {
-    // N = 128: double-buffered input stages, Y accumulators and S^T; the chunk state
-    // accumulates in the half of the score buffer that the packed G' leaves free.
-    // N = 256: the wider state takes the room of the second buffers.
+    // N = 128: double-buffered input stages and S^T. N = 256: one of each (the wider B, C and
+    // S^T fill shared memory).
     static constexpr bool kWide = N == 256;
     static constexpr int kStages = kWide ? 1 : 2;
-    static constexpr int kYBufs = kWide ? 1 : 2;
+    static constexpr int kYBufs = 2;
     static constexpr int kStBufs = kWide ? 1 : 2;
-    static constexpr bool kDsInG = !kWide;
     static constexpr int kPanels = N / 64;           // 64-column panels of B and C
     static constexpr int kPanelBytes = kQ * 128;     // 128 rows x 128 B
     static constexpr int kCBytes = kPanels * kPanelBytes;
@@ -74,22 +74,27 @@ struct Cfg {
     static constexpr int kOffXp = kStages * kStageBytes;
     static constexpr int kOffSt = kOffXp + kXBytes;
     static constexpr int kOffSmall = kOffSt + kStBufs * kStBytes;
-    // per stage: dt, A_cs (log2 domain) and the block scalars {A_cs[127], m, exact?, valid tokens}
+    // per stage: dt, A_cs (log2 domain), the block scalars {A_cs[127], m, exact?, valid tokens}
+    // and the block's coordinates {b, h, c, last of its piece}; they travel with the x tile
     static constexpr int kOffDts = kOffSmall;                       // float [kStages][128]
     static constexpr int kOffAcs = kOffDts + kStages * kQ * 4;      // float [kStages][128]
     static constexpr int kOffBlk = kOffAcs + kStages * kQ * 4;      // float4 [kStages]
-    static constexpr int kOffCrd = kOffBlk + kStages * 16;          // int4 [kStages]: b, h, c, last-of-piece
+    static constexpr int kOffCrd = kOffBlk + kStages * 16;          // int4 [kStages]
     static constexpr int kOffBar = kOffCrd + kStages * 16;          // uint64 barriers
-    static constexpr int kNumBars = 3 * kStages + 11 + kStBufs + 2 * kYBufs;
+    // TMEM columns: score buffers j at 128 j (fp32 C B^T, then G' packed in its first 64);
+    // Y buffers at 256 + 64 i; the chunk-state accumulators (64 columns per 128 state rows)
+    // from 384, two of them for N = 128 and one for N = 256.
+    static constexpr int kTmY = 256;
+    static constexpr int kTmDs = 384;
+    static constexpr int kDsCols = N / 2;
+    static constexpr int kDsBufs = 128 / kDsCols;
+    static constexpr int kTmCols = 512;
+    static constexpr int kNumBars = 5 * kStages + 6 + 2 * kDsBufs + kStBufs + 2 * kYBufs + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;         // tmem base, abort flag
     static constexpr int kSmemBytes = kOffMisc + 16;
     static constexpr int kSmemAlloc = kSmemBytes + 1024;            // slack for 1024-B alignment
-    // TMEM columns: score buffers j at 128 j; Y buffer i at 256 + 128 i (Y_diag, then Y_off
-    // at +64); the chunk state inside score buffer j at 128 j + 64, or (wide) at 384.
-    static constexpr int kTmY = 256;
-    static constexpr int kTmCols = 512;
     static_assert(kSmemAlloc <= 232448, "shared memory budget");
-    static constexpr uint32_t kTxBytes = kStageBytes;
+    static constexpr uint32_t kTxBC = 2 * kCBytes, kTxX = kXBytes;
 };
 
 struct Params {
@@ -340,7 +345,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return r;
 }
 // Packed fp32 pairs (sm_100): s = g s + d r on two lanes of the state at once, and
-// the epilogue's el * ys + rd * yd on two columns at once.
+// w (a, b) rounded to a bf16 pair.
 __device__ __forceinline__ void fma2_state(float &s0, float &s1, float g, float d, uint32_t r0, uint32_t r1) {
     asm("{\n\t.reg .b64 s, q, gg, dd;\n\t"
         "mov.b64 s, {%0, %1};\n\tmov.b64 q, {%4, %5};\n\t"
@@ -350,16 +355,14 @@ __device__ __forceinline__ void fma2_state(float &s0, float &s1, float g, float 
         : "+f"(s0), "+f"(s1)
         : "f"(g), "f"(d), "r"(r0), "r"(r1));
 }
-__device__ __forceinline__ uint32_t epi2_bf16(float el, float rd, uint32_t ys0, uint32_t ys1, uint32_t yd0,
-                                              uint32_t yd1) {
+__device__ __forceinline__ uint32_t scale2_bf16(float w, float a, float b) {
     uint32_t o;
-    asm("{\n\t.reg .b64 a, b, e, r;\n\t.reg .f32 lo, hi;\n\t"
-        "mov.b64 a, {%3, %4};\n\tmov.b64 b, {%5, %6};\n\t"
-        "mov.b64 e, {%1, %1};\n\tmov.b64 r, {%2, %2};\n\t"
-        "mul.rn.f32x2 b, b, r;\n\tfma.rn.f32x2 a, e, a, b;\n\t"
-        "mov.b64 {lo, hi}, a;\n\tcvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
+    asm("{\n\t.reg .b64 v, ww;\n\t.reg .f32 lo, hi;\n\t"
+        "mov.b64 v, {%2, %3};\n\tmov.b64 ww, {%1, %1};\n\t"
+        "mul.rn.f32x2 v, v, ww;\n\t"
+        "mov.b64 {lo, hi}, v;\n\tcvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
         : "=r"(o)
-        : "f"(el), "f"(rd), "r"(ys0), "r"(ys1), "r"(yd0), "r"(yd1));
+        : "f"(w), "f"(a), "f"(b));
     return o;
 }
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
@@ -433,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_ssd_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
              const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y, const Params prm) {
     using Cf = Cfg<N>;
-    constexpr int S = Cf::kStages, YB = Cf::kYBufs, SB = Cf::kStBufs;
+    constexpr int S = Cf::kStages, YB = Cf::kYBufs, SB = Cf::kStBufs, DB = Cf::kDsBufs;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -443,18 +446,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     float4 *blk_s = reinterpret_cast<float4 *>(sm + Cf::kOffBlk);
     int4 *crd_s = reinterpret_cast<int4 *>(sm + Cf::kOffCrd);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + Cf::kOffBar);
-    uint64_t *full = bar;                // [S]   stage loaded (TMA bytes + dt)
-    uint64_t *empty = full + S;          // [S]   stage consumed: 4 issuer commits + 4 T warps + 4 E warps
-    uint64_t *gfull = empty + S;         // [2]   C B^T in score buffer j
-    uint64_t *gp = gfull + 2;            // [2]   G' written back to score buffer j, and X'' (T)
-    uint64_t *xpr = gp + 2;              // [S]   X'' of stage k written (T)
-    uint64_t *dsdone = xpr + S;          // [2]   chunk state of block t done, buffer t % 2
-    uint64_t *dsfree = dsdone + 2;       // [2]   chunk state of block t read by E
-    uint64_t *ydd = dsfree + 2;          // [2]   Y_diag of block t done (score buffer t % 2 reusable)
-    uint64_t *sready = ydd + 2;          // [SB]  S_in^T of block t written (E)
-    uint64_t *yfull = sready + SB;       // [YB]  Y_diag and Y_off of block t done
+    uint64_t *full_bc = bar;             // [S]   B and C of stage k loaded
+    uint64_t *full_x = full_bc + S;      // [S]   x of stage k loaded and its step-0 values written
+    uint64_t *empty_bc = full_x + S;     // [S]   B, C consumed: C B^T, chunk-state and Y_off commits
+    uint64_t *empty_x = empty_bc + S;    // [S]   x and step-0 values consumed: 4 T + 4 E warps, 2 commits
+    uint64_t *xpr = empty_x + S;         // [S]   X'' of stage k written (T)
+    uint64_t *gfull = xpr + S;           // [2]   C B^T in score buffer j
+    uint64_t *gp = gfull + 2;            // [2]   G' written back to score buffer j (T)
+    uint64_t *ydd = gp + 2;              // [2]   Y_diag of block t done (score buffer t % 2 reusable)
+    uint64_t *dsdone = ydd + 2;          // [DB]  chunk state of block t done
+    uint64_t *dsfree = dsdone + DB;      // [DB]  chunk state of block t read by E
+    uint64_t *sready = dsfree + DB;      // [SB]  S_in^T of block t written (E)
+    uint64_t *yfull = sready + SB;       // [YB]  Y of block t done
     uint64_t *yfree = yfull + YB;        // [YB]  Y of block t read by E
-    uint64_t *fin = yfree + YB;          // [1]   every MMA of this CTA done (4 issuers)
+    uint64_t *fin = yfree + YB;          // [1]   every MMA of this CTA done (3 issuers)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + Cf::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + Cf::kOffMisc + 4);
     int *status = prm.status;
@@ -467,23 +472,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 4 + 4 + 4);
+            mbar_init(&full_bc[i], 1);
+            mbar_init(&full_x[i], 1);
+            mbar_init(&empty_bc[i], 3);
+            mbar_init(&empty_x[i], 4 + 4 + 2);
+            mbar_init(&xpr[i], 128);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&gfull[i], 1);
             mbar_init(&gp[i], 128);
-            mbar_init(&dsdone[i], 1);
-            mbar_init(&dsfree[i], 128);
             mbar_init(&ydd[i], 1);
         }
-        for (int i = 0; i < S; ++i) mbar_init(&xpr[i], 128);
+        for (int i = 0; i < DB; ++i) {
+            mbar_init(&dsdone[i], 1);
+            mbar_init(&dsfree[i], 128);
+        }
         for (int i = 0; i < SB; ++i) mbar_init(&sready[i], 128);
         for (int i = 0; i < YB; ++i) {
-            mbar_init(&yfull[i], 2);
+            mbar_init(&yfull[i], 1);
             mbar_init(&yfree[i], 128);
         }
-        mbar_init(fin, 4);
+        mbar_init(fin, 3);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -504,17 +513,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto stage_x = [&](int k) { return sm + k * Cf::kStageBytes + 2 * Cf::kCBytes; };
     unsigned char *xp = sm + Cf::kOffXp;
     auto st_buf = [&](int i) { return sm + Cf::kOffSt + i * Cf::kStBytes; };
-    // TMEM column of the chunk state of task t
-    auto ds_col = [&](int t) -> uint32_t { return Cf::kDsInG ? 128u * (uint32_t)(t & 1) + 64u : 384u; };
+    // TMEM column of the chunk-state accumulator of task t
+    auto ds_col = [&](int t) -> uint32_t { return (uint32_t)(Cf::kTmDs + Cf::kDsCols * (t % DB)); };
     constexpr uint32_t kIdG = idesc(128, 128, false, false);
     constexpr uint32_t kIdDs = idesc(128, 64, true, true);
     constexpr uint32_t kIdY = idesc(128, 64, false, true);
 
     if (warp == kWarpTma) {
-        // ------------------------------------------------------------- loads, step 0, Y_diag issue
-        // Task t's stage is loaded, then Y_diag of task t-1 is issued (with one stage, Y_diag of
-        // t-1 goes first: the stage of t is released only once Y_diag of t-1 is done), then step 0
-        // of task t+1 runs on dt that was fetched one task earlier, and dt of task t+2 is fetched.
+        // ------------------------------------------------------------- loads and step 0
+        // B and C of task t are loaded as soon as their stage is free, then x with the step-0
+        // values; step 0 of task t+1 then runs on dt that was fetched one task earlier, and dt
+        // of task t+2 is fetched.
         const uint64_t pol_keep = policy_evict_last(), pol_stream = policy_evict_first();
         // Lane i handles tokens 4 i .. 4 i + 3 of a block.
         float raw[4], a_raw = 0.f;  // dt and A_h of the task after the prepared one
@@ -582,36 +591,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool factored = __all_sync(0xffffffffu, dt_ok) && (mx - mn <= 128.f);
             blkn = make_float4(tot, factored ? 0.5f * (mx + mn) : tot, factored ? 0.f : 1.f, (float)nvalid_raw);
         };
-        auto issue_yd = [&](int t) -> bool {  // Y_diag = G' X'' with G' in TMEM   (M = l, N = p, K = s)
-            const int k = t % S, j = t & 1, yb = t % YB;
-            if (!wait_warp(&gp[j], (uint32_t)(t >> 1) & 1u, abort_flag, status)) return false;
-            if (t >= YB && !wait_warp(&yfree[yb], (uint32_t)((t - YB) / YB) & 1u, abort_flag, status)) return false;
-            if (lane == 0) {
-                tc_fence_after();
-                const uint32_t xa = smem_u32(stage_x(k));  // X'' in place (x itself in the exact form)
-#pragma unroll 1
-                for (int kk = 0; kk < kQ / 16; ++kk)
-                    mma_ts(tmem + Cf::kTmY + 128 * yb, tmem + 128 * j + 8 * kk, sdesc(xa + kk * 2048, 1024, 1024),
-                           kIdY, kk > 0);
-                mma_commit(&yfull[yb]);
-                mma_commit(&ydd[j]);
-                mma_commit(&empty[k]);
-            }
-            __syncwarp();
-            return true;
-        };
         if (ntask > 0) {
             fetch(0);
             prep();
             if (ntask > 1) fetch(1);
         }
-        int nl = 0;
-        bool ok = true;
-        for (int t = 0; ok && t < ntask; ++t) {
+        int nbc = 0, nx = 0;  // loads issued
+        for (int t = 0; t < ntask; ++t) {
             const int k = t % S;
-            if (S == 1 && t >= 1 && !(ok = issue_yd(t - 1))) break;
-            if (t >= S && !(ok = wait_warp(&empty[k], (uint32_t)((t / S) - 1) & 1u, abort_flag, status))) break;
-            const int b = crd_n.x, h = crd_n.y, c = crd_n.z;
+            const uint32_t ph = (uint32_t)((t / S) - 1) & 1u;
+            const int b = crd_n.x, h = crd_n.y, c = crd_n.z, t0 = c * kQ, g = h / hpg;
+            if (t >= S && !wait_warp(&empty_bc[k], ph, abort_flag, status)) break;
+            if (lane == 0) {
+                mbar_arrive_tx(&full_bc[k], Cf::kTxBC);
+                for (int pn = 0; pn < Cf::kPanels; ++pn) {
+                    tma_load_4d_hint(stage_c(k) + pn * Cf::kPanelBytes, &tm_c, &full_bc[k], 64 * pn, g, t0, b, pol_keep);
+                    tma_load_4d_hint(stage_b(k) + pn * Cf::kPanelBytes, &tm_b, &full_bc[k], 64 * pn, g, t0, b, pol_keep);
+                }
+            }
+            nbc = t + 1;
+            if (t >= S && !wait_warp(&empty_x[k], ph, abort_flag, status)) break;
             reinterpret_cast<float4 *>(dts + k * kQ)[lane] = dtn;
             reinterpret_cast<float4 *>(acs_s + k * kQ)[lane] = acn;
             if (lane == 0) {
@@ -620,29 +619,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
             if (lane == 0) {
-                const int t0 = c * kQ, g = h / hpg;
-                mbar_arrive_tx(&full[k], Cf::kTxBytes);
-                for (int pn = 0; pn < Cf::kPanels; ++pn) {
-                    tma_load_4d_hint(stage_c(k) + pn * Cf::kPanelBytes, &tm_c, &full[k], 64 * pn, g, t0, b, pol_keep);
-                    tma_load_4d_hint(stage_b(k) + pn * Cf::kPanelBytes, &tm_b, &full[k], 64 * pn, g, t0, b, pol_keep);
-                }
-                tma_load_4d_hint(stage_x(k), &tm_x, &full[k], 0, h, t0, b, pol_stream);
+                mbar_arrive_tx(&full_x[k], Cf::kTxX);
+                tma_load_4d_hint(stage_x(k), &tm_x, &full_x[k], 0, h, t0, b, pol_stream);
             }
             __syncwarp();
-            nl = t + 1;
-            if (S > 1 && t >= 1 && !(ok = issue_yd(t - 1))) break;
+            nx = t + 1;
             if (t + 1 < ntask) {
                 prep();
                 if (t + 2 < ntask) fetch(t + 2);
             }
         }
-        if (ok && ntask > 0) issue_yd(ntask - 1);
-        if (lane == 0) mma_commit(fin);
         // drain: loads still in flight land before the CTA exits
         if (lane == 0) {
-            for (int t = max(0, nl - S); t < nl; ++t) {
-                const unsigned long long t0 = now_ns();
-                while (!mbar_try(&full[t % S], (uint32_t)(t / S) & 1u) && now_ns() - t0 < kWaitNs) {
+            for (int t = max(0, nbc - S); t < nbc; ++t) {
+                const unsigned long long w0 = now_ns();
+                while (!mbar_try(&full_bc[t % S], (uint32_t)(t / S) & 1u) && now_ns() - w0 < kWaitNs) {
+                }
+            }
+            for (int t = max(0, nx - S); t < nx; ++t) {
+                const unsigned long long w0 = now_ns();
+                while (!mbar_try(&full_x[t % S], (uint32_t)(t / S) & 1u) && now_ns() - w0 < kWaitNs) {
                 }
             }
         }
@@ -652,12 +648,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             for (int t = 0; t < ntask; ++t) {
                 const int k = t % S, j = t & 1;
-                if (!wait_phase(&full[k], (uint32_t)(t / S) & 1u, abort_flag, status)) break;
-                if (t >= 2) {  // score buffer j: G' of task t-2 consumed, its chunk state read
-                    if (!wait_phase(&ydd[j], (uint32_t)((t - 2) >> 1) & 1u, abort_flag, status)) break;
-                    if (Cf::kDsInG && !wait_phase(&dsfree[j], (uint32_t)((t - 2) >> 1) & 1u, abort_flag, status))
-                        break;
-                }
+                if (!wait_phase(&full_bc[k], (uint32_t)(t / S) & 1u, abort_flag, status)) break;
+                // score buffer j: G' of task t-2 consumed by its Y_diag
+                if (t >= 2 && !wait_phase(&ydd[j], (uint32_t)((t - 2) >> 1) & 1u, abort_flag, status)) break;
                 tc_fence_after();
                 const uint32_t ca = smem_u32(stage_c(k)), ba = smem_u32(stage_b(k));
 #pragma unroll 1
@@ -666,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_ss(tmem + 128 * j, sdesc(ca + off, 16, 1024), sdesc(ba + off, 16, 1024), kIdG, kk > 0);
                 }
                 mma_commit(&gfull[j]);
-                mma_commit(&empty[k]);
+                mma_commit(&empty_bc[k]);
             }
             mma_commit(fin);
         }
@@ -675,13 +668,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------- dS^T = B^T X''   (M = n, N = p, K = s)
         if (lane == 0) {
             for (int t = 0; t < ntask; ++t) {
-                const int k = t % S, j = t & 1;
+                const int k = t % S, db = t % DB;
                 if (!wait_phase(&xpr[k], (uint32_t)(t / S) & 1u, abort_flag, status)) break;
-                if (Cf::kDsInG) {  // T is done reading C B^T from the half this state goes to
-                    if (!wait_phase(&gp[j], (uint32_t)(t >> 1) & 1u, abort_flag, status)) break;
-                } else if (t >= 1) {
-                    if (!wait_phase(&dsfree[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u, abort_flag, status)) break;
-                }
+                if (!wait_phase(&full_bc[k], (uint32_t)(t / S) & 1u, abort_flag, status)) break;
+                if (t >= DB && !wait_phase(&dsfree[db], (uint32_t)((t - DB) / DB) & 1u, abort_flag, status)) break;
                 tc_fence_after();
                 // X'' in place in the stage, or (exact form) X' in its own buffer
                 const bool exact = blk_s[k].z != 0.f;
@@ -694,30 +684,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                                sdesc(ba + 2 * hf * Cf::kPanelBytes + kk * 2048, Cf::kPanelBytes, 1024),
                                sdesc(xa + kk * 2048, Cf::kPanelBytes, 1024), kIdDs, kk > 0);
                 }
-                mma_commit(&dsdone[j]);
-                mma_commit(&empty[k]);
+                mma_commit(&dsdone[db]);
+                mma_commit(&empty_bc[k]);
+                mma_commit(&empty_x[k]);
             }
             mma_commit(fin);
         }
         __syncwarp();
     } else if (warp == kWarpYs) {
-        // ------------------------------------------------------------- Y_off = C S_in^T   (M = l, N = p, K = n)
+        // ------------------------------------------------------------- Y = C (s S_in)^T + G' X''
+        // One accumulator: Y_off first (M = l, N = p, K = n), then Y_diag (K = s) with G' as the
+        // TMEM A operand. In the factored form s = exp(m) and y = exp(A_cs[l] - m) Y; in the exact
+        // form T has scaled the rows of C by exp(A_cs[l]), s = 1 and y = Y.
         if (lane == 0) {
             for (int t = 0; t < ntask; ++t) {
-                const int k = t % S, yb = t % YB;
+                const int k = t % S, j = t & 1, yb = t % YB;
+                const uint32_t yacc = tmem + Cf::kTmY + 64 * yb;
+                if (!wait_phase(&full_bc[k], (uint32_t)(t / S) & 1u, abort_flag, status)) break;
                 if (!wait_phase(&sready[t % SB], (uint32_t)(t / SB) & 1u, abort_flag, status)) break;
-                if (!wait_phase(&full[k], (uint32_t)(t / S) & 1u, abort_flag, status)) break;
                 if (t >= YB && !wait_phase(&yfree[yb], (uint32_t)((t - YB) / YB) & 1u, abort_flag, status)) break;
+                const bool exact = blk_s[k].z != 0.f;  // written before S_in^T of task t was
+                if (exact && !wait_phase(&gp[j], (uint32_t)(t >> 1) & 1u, abort_flag, status)) break;
                 tc_fence_after();
                 const uint32_t ca = smem_u32(stage_c(k)), sa = smem_u32(st_buf(t % SB));
 #pragma unroll 1
                 for (int kk = 0; kk < N / 16; ++kk) {
                     const uint32_t off = (uint32_t)((kk >> 2) * Cf::kPanelBytes + (kk & 3) * 32);
-                    mma_ss(tmem + Cf::kTmY + 128 * yb + 64, sdesc(ca + off, 16, 1024), sdesc(sa + kk * 2048, 1024, 1024),
-                           kIdY, kk > 0);
+                    mma_ss(yacc, sdesc(ca + off, 16, 1024), sdesc(sa + kk * 2048, 1024, 1024), kIdY, kk > 0);
                 }
+                mma_commit(&empty_bc[k]);
+                if (!exact && !wait_phase(&gp[j], (uint32_t)(t >> 1) & 1u, abort_flag, status)) break;
+                tc_fence_after();
+                const uint32_t xa = smem_u32(stage_x(k));  // X'' in place (x itself in the exact form)
+#pragma unroll 1
+                for (int kk = 0; kk < kQ / 16; ++kk)
+                    mma_ts(yacc, tmem + 128 * j + 8 * kk, sdesc(xa + kk * 2048, 1024, 1024), kIdY, 1);
                 mma_commit(&yfull[yb]);
-                mma_commit(&empty[k]);
+                mma_commit(&ydd[j]);
+                mma_commit(&empty_x[k]);
             }
             mma_commit(fin);
         }
@@ -742,7 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         for (int t = 0; t < ntask; ++t) {
             const int k = t % S, j = t & 1;
-            if (!wait_warp(&full[k], (uint32_t)(t / S) & 1u, abort_flag, status)) break;
+            if (!wait_warp(&full_x[k], (uint32_t)(t / S) & 1u, abort_flag, status)) break;
             const float Dh = prm.D ? __ldg(prm.D + crd_s[k].y) : 0.f;
             const float *dk = dts + k * kQ;
             const float *acsW = acs_s + k * kQ;
@@ -753,7 +757,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // X''[row,:] = exp(m - A_cs[row]) dt_row x_row, in place; in the exact form (m = A_cs[127])
             // into its own buffer, once the previous chunk-state MMA is done reading that
             if (exact && t > 0 &&
-                !wait_warp(&dsdone[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u, abort_flag, status))
+                !wait_warp(&dsdone[(t - 1) % DB], (uint32_t)((t - 1) / DB) & 1u, abort_flag, status))
                 break;
             scale_row(stage_x(k), exact ? xp : stage_x(k), ex2(blk.y - acs_r) * dt_r);
             fence_proxy_async();
@@ -795,12 +799,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int jb = qtr + 1; jb < 4; ++jb) tmem_st16(gaddr + 16 * jb, zero);
             } else {
                 gprime_exact(gaddr, qtr, row, acs_r, acsW, dk, Dh);
+                // C[row,:] *= exp(A_cs[row]) in place (C B^T is done with C): the row factor of
+                // Y_off, which the exact form cannot share with Y_diag
+                if (!wait_warp(&full_bc[k], (uint32_t)(t / S) & 1u, abort_flag, status)) break;
+                const float el = ex2(acs_r);
+                unsigned char *cs = stage_c(k);
+#pragma unroll 1
+                for (int pn = 0; pn < Cf::kPanels; ++pn) scale_row(cs + pn * Cf::kPanelBytes, cs + pn * Cf::kPanelBytes, el);
+                fence_proxy_async();
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&gp[j]);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[k]);  // this warp is done with the stage
+            if (lane == 0) mbar_arrive(&empty_x[k]);  // this warp is done with x and the step-0 values
         }
     } else {
         // ------------------------------------------------------------- E: state chain + epilogue
@@ -809,7 +821,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_off = (uint32_t)(qtr * 32) << 16;
         constexpr int NH = N / 128;  // state rows per thread: n = row + 128 i
         float Sr[NH][kP];
-        auto write_st = [&](int t) {  // S_in^T of task t, bf16, into its buffer
+        // S_in^T of task t, bf16, scaled by s = exp(m) of task t in the factored form (1 in the
+        // exact form), into its buffer
+        auto write_st = [&](int t) -> bool {
+            if (!wait_warp(&full_x[t % S], (uint32_t)(t / S) & 1u, abort_flag, status)) return false;
+            const float4 bt = blk_s[t % S];
+            const float sg = bt.z != 0.f ? 1.f : ex2(bt.y);
             unsigned char *stb = st_buf(t % SB);
             // the buffer doubles as this warp's y staging slice: its last y store must have read it
             if (lane == 0) bulk_wait_read();
@@ -820,15 +837,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
                     uint4 o;
-                    o.x = pack_bf16(Sr[i][8 * ch + 0], Sr[i][8 * ch + 1]);
-                    o.y = pack_bf16(Sr[i][8 * ch + 2], Sr[i][8 * ch + 3]);
-                    o.z = pack_bf16(Sr[i][8 * ch + 4], Sr[i][8 * ch + 5]);
-                    o.w = pack_bf16(Sr[i][8 * ch + 6], Sr[i][8 * ch + 7]);
+                    o.x = scale2_bf16(sg, Sr[i][8 * ch + 0], Sr[i][8 * ch + 1]);
+                    o.y = scale2_bf16(sg, Sr[i][8 * ch + 2], Sr[i][8 * ch + 3]);
+                    o.z = scale2_bf16(sg, Sr[i][8 * ch + 4], Sr[i][8 * ch + 5]);
+                    o.w = scale2_bf16(sg, Sr[i][8 * ch + 6], Sr[i][8 * ch + 7]);
                     *reinterpret_cast<uint4 *>(stb + swz(n, ch)) = o;
                 }
             }
             fence_proxy_async();
             mbar_arrive(&sready[t % SB]);
+            return true;
         };
         // Initial state of the piece that starts at task t: h0 (or zeros) at the start of a
         // stream, otherwise the state handed over by the previous CTA.
@@ -874,19 +892,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 atomicAdd(prm.flags + blockIdx.x, 1);
             }
         };
-        bool ok = ntask > 0 && load_init(0);
-        if (ok) write_st(0);
+        bool ok = ntask > 0 && load_init(0) && write_st(0);
         for (int t = 0; ok && t < ntask; ++t) {
-            const int k = t % S, j = t & 1, yb = t % YB;
-            if (!(ok = wait_warp(&full[k], (uint32_t)(t / S) & 1u, abort_flag, status))) break;
+            const int k = t % S, yb = t % YB, db = t % DB;
+            if (!(ok = wait_warp(&full_x[k], (uint32_t)(t / S) & 1u, abort_flag, status))) break;
             const int4 crd = crd_s[k];  // {b, h, c, last of its piece}
             const int h = crd.y, c = crd.z;
             const float4 blk = blk_s[k];  // {A_cs[127], m, exact?, valid tokens}
             const float acs_r = acs_s[k * kQ + row];
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[k]);  // done with the step-0 values of the stage
+            if (lane == 0) mbar_arrive(&empty_x[k]);  // done with the step-0 values of the stage
             // step 3: S <- exp(A_cs[127]) S + exp(A_cs[127] - m) dS
-            if (!(ok = wait_warp(&dsdone[j], (uint32_t)(t >> 1) & 1u, abort_flag, status))) break;
+            if (!(ok = wait_warp(&dsdone[db], (uint32_t)(t / DB) & 1u, abort_flag, status))) break;
             tc_fence_after();
             {
                 const float gam = ex2(blk.x), dsc = ex2(blk.x - blk.y);
@@ -903,7 +920,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 tc_fence_before();
-                mbar_arrive(&dsfree[j]);
+                mbar_arrive(&dsfree[db]);
             }
             const bool last_of_piece = crd.w != 0;
             if (last_of_piece) store_final(t);
@@ -911,24 +928,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Y_off of task t-1, which is done (the epilogue of t-1 waited for it).
             if (SB == 2 && t + 1 < ntask) {
                 if (last_of_piece && !(ok = load_init(t + 1))) break;
-                write_st(t + 1);
+                if (!(ok = write_st(t + 1))) break;
             }
-            // epilogue: y = exp(A_cs[l] - m) Y_diag + exp(A_cs[l]) Y_off   (D x is inside Y_diag;
-            // the exact form has no row factor)
+            // epilogue: y = exp(A_cs[l] - m) Y in the factored form, y = Y in the exact form (D x is
+            // inside Y)
             if (!(ok = wait_warp(&yfull[yb], (uint32_t)(t / YB) & 1u, abort_flag, status))) break;
             tc_fence_after();
             {
                 // y rows of this warp (32 tokens x 64 values) are staged, 128-byte swizzled, in its
                 // 4 KB slice of the S^T buffer of task t (free: Y_off of task t is done) and written
                 // by one bulk tensor store.
-                const float el = ex2(acs_r), rd = blk.z != 0.f ? 1.f : ex2(acs_r - blk.y);
+                const float rd = blk.z != 0.f ? 1.f : ex2(acs_r - blk.y);
                 unsigned char *stage_y = st_buf(t % SB);
-                const uint32_t ya = tmem + Cf::kTmY + 128 * yb + lane_off;
+                const uint32_t ya = tmem + Cf::kTmY + 64 * yb + lane_off;
 #pragma unroll 1
                 for (int qq = 0; qq < 4; ++qq) {  // 16 columns at a time
-                    uint32_t yd[16], ys[16];
-                    tmem_ld16(ya + 16 * qq, yd);
-                    tmem_ld16(ya + 64 + 16 * qq, ys);
+                    uint32_t yv[16];
+                    tmem_ld16(ya + 16 * qq, yv);
                     tmem_wait_ld();
                     if (qq == 3) {
                         tc_fence_before();
@@ -936,7 +952,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     uint32_t o[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) o[e] = epi2_bf16(el, rd, ys[2 * e], ys[2 * e + 1], yd[2 * e], yd[2 * e + 1]);
+                    for (int e = 0; e < 8; ++e) o[e] = scale2_bf16(rd, __uint_as_float(yv[2 * e]), __uint_as_float(yv[2 * e + 1]));
                     *reinterpret_cast<uint4 *>(stage_y + swz(row, 2 * qq)) = make_uint4(o[0], o[1], o[2], o[3]);
                     *reinterpret_cast<uint4 *>(stage_y + swz(row, 2 * qq + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
                 }
@@ -952,7 +968,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // with one S^T buffer it is free only now (Y_off of task t is done)
             if (SB == 1 && t + 1 < ntask) {
                 if (last_of_piece && !(ok = load_init(t + 1))) break;
-                write_st(t + 1);
+                if (!(ok = write_st(t + 1))) break;
             }
         }
     }
