@@ -37,6 +37,24 @@ def peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ssd_fwd_tc_mamba2_2p7b_traffic.json")
+TC_SOURCE = os.path.join(ROOT, "state_space_sequence_chunked_b200", "csrc", "ssd_tc.cu")
+
+
+def measured_traffic(wl, path):
+    """DRAM bytes (read + write) per launch of the tensor-core kernel from the committed ncu
+    capture, if that capture was taken of the kernel source as it is now; else None."""
+    import hashlib
+
+    if wl.name != "mamba2_2p7b" or path != "tcgen05" or not os.path.exists(TRAFFIC_FILE):
+        return None
+    rec = json.load(open(TRAFFIC_FILE))
+    src = hashlib.sha256(open(TC_SOURCE, "rb").read()).hexdigest()
+    if rec.get("source_sha256") != src:
+        return None
+    return rec["dram_read_bytes"] + rec["dram_write_bytes"]
+
+
 def algorithmic(wl):
     """Bytes each input is read once + outputs written once; FLOPs of the chunked
     method with the structurally-zero upper triangle of the diagonal blocks skipped
@@ -123,7 +141,9 @@ class ClockSampler:
         return out
 
 
-def dist_setup():
+def dist_setup(backend: str = "nccl"):
+    """Rank, world size and local rank from the launcher's environment; for N > 1 a
+    process group (NCCL over the GPUs; gloo on CPU for the host-logic tests)."""
     import torch
     import torch.distributed as dist
 
@@ -133,21 +153,30 @@ def dist_setup():
     if ws > 1:
         import datetime
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=180)
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timeout)
     return ws, rank, local
 
 
-def reduce_max(v: float, ws: int) -> float:
+def reduce_max(v: float, ws: int, device: str = "cuda") -> float:
+    """Max over ranks (the job's time is the slowest rank's)."""
     if ws == 1:
         return v
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([v], device="cuda", dtype=torch.float64)
+    t = torch.tensor([v], device=device, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(wl, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling: per-rank work is fixed)."""
+    return wl.seed + 1000 * rank
 
 
 def barrier(ws):
@@ -227,6 +256,88 @@ def reference_arm(args, wl):
     return 0
 
 
+
+VERIFY_METRIC = "SSD speculative verify + state selection draft tokens/s (batch*K/s)"
+
+
+def verify_main(args, wl):
+    """One step = ssd_verify (K draft tokens from a saved state, every state written) and
+    ssd_select_state (keep the state at the accepted index), on seeded inputs in HBM."""
+    import torch
+
+    from state_space_sequence_chunked_b200 import _binding as ssd
+    from state_space_sequence_chunked_b200 import inputs
+
+    ws, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    d = inputs.draw(wl, seed=rank_seed(wl, rank))
+    g = {k: d[k].torch(dev) for k in ("x", "dt", "A", "B", "C", "D", "h0")}
+    acc = torch.from_numpy(d["accepted"]).to(dev)
+    Bsz, K, H, P, N, G = wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.dstate, wl.ngroups
+    so = torch.empty(Bsz, K, H, P, N, device=dev)
+    y = torch.empty_like(g["x"])
+    keep = torch.empty(Bsz, H, P, N, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ssd.ssd_verify(g["h0"], g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], states_out=so, y=y, stream=stream)
+        ssd.ssd_select_state(g["h0"], so, acc, h_keep=keep, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev)
+    clocks.start()
+    ev0, ev1, ev2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    barrier(ws)
+    torch.cuda.synchronize()
+    clocks.mark_start()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark_end()
+    barrier(ws)
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    # the verify kernel alone, for its own roofline
+    ev0.record(stream)
+    for _ in range(args.steps):
+        ssd.ssd_verify(g["h0"], g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], states_out=so, y=y, stream=stream)
+    ev2.record(stream)
+    torch.cuda.synchronize()
+    ms_v = ev0.elapsed_time(ev2) / args.steps
+    ms_max = reduce_max(ms, ws)
+    e = 2  # bf16 inputs
+    v_bytes = (Bsz * H * P * N * 4 * (1 + K) + Bsz * K * H * P * e * 2 + Bsz * K * H * e
+               + 2 * Bsz * K * G * N * e + 2 * H * 4)
+    s_bytes = 2 * Bsz * H * P * N * 4 + Bsz * 4
+    hbm, _, src = peaks()
+    tokens = Bsz * K
+    if rank == 0:
+        line = {
+            "metric": VERIFY_METRIC, "value": tokens * ws / (ms_max * 1e-3), "unit": "tokens/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "batch": Bsz, "K": K, "nheads": H, "headdim": P, "dstate": N,
+                       "ngroups": G, "l2": "states_out 1074 MB per step vs 126 MB L2; no flush"},
+            "roofline": {"bound": "hbm", "achieved": v_bytes / (ms_v * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                         "frac": v_bytes / (ms_v * 1e-3) / 1e9 / hbm, "traffic": None, "kernel": "k_verify",
+                         "peak_source": src, "alg_bytes": v_bytes, "ms": ms_v,
+                         "step_bytes": v_bytes + s_bytes,
+                         "step_frac": (v_bytes + s_bytes) / (ms * 1e-3) / 1e9 / hbm},
+            "cpu_baseline": None, "gpu_launches": 2 * args.steps, "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
 # ---------------------------------------------------------------------------------------
 
 def main():
@@ -244,7 +355,9 @@ def main():
 
     wl = inputs.WORKLOADS[args.workload]
     if wl.verify:
-        raise SystemExit("bench.py times the forward workloads")
+        if args.impl == "reference":
+            raise SystemExit("the reference arm times the forward workloads")
+        return verify_main(args, wl)
     if args.impl == "reference":
         return reference_arm(args, wl)
 
@@ -255,7 +368,7 @@ def main():
     ws, rank, local = dist_setup()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    d = inputs.draw(wl, seed=wl.seed + 1000 * rank)
+    d = inputs.draw(wl, seed=rank_seed(wl, rank))
     code = ssd.SSD_BF16 if wl.dtype == "bf16" else ssd.SSD_F32
     plan = ssd.fwd_plan(wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.ngroups, wl.dstate, code, wl.chunk)
     g = {k: d[k].torch(dev) for k in ("x", "dt", "A", "B", "C", "D")}
@@ -351,8 +464,10 @@ def main():
                        "path": plan["path"], "per_rank_batch": wl.batch,
                        "l2": "inputs larger than L2 (x and y 335.5 MB each per step vs 126 MB L2); no flush"},
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                         "frac": achieved / peak, "traffic": None,
-                         "kernel": "whole ssd_fwd call (%d launches)" % plan["kernels"],
+                         "frac": achieved / peak, "traffic": measured_traffic(wl, plan["path"]),
+                         "kernel": ("k_ssd_tc<%d> (the whole call: one launch after a status-word memset)" % wl.dstate
+                                    if plan["path"] == "tcgen05" else
+                                    "whole ssd_fwd call (%d launches)" % plan["kernels"]),
                          "peak_source": src, "alg_bytes": nbytes, "alg_flops": flops,
                          "roofline_tokens_per_s": tokens / t_roof, "frac_of_roofline_time": t_roof / (ms * 1e-3)},
             "cpu_baseline": cpu,
