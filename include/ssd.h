@@ -155,9 +155,10 @@ ssd_status_t ssd_fwd_static_scratch(const ssd_shape_t *shape, ssd_dtype_t dtype,
  *   dt          [B, K, H]         dtype
  *   A, D        [H]               fp32 (D may be NULL = 0)
  *   Bm, Cm      [B, K, G, N]      dtype
- *   states_out  [B, K, H, P, N]   fp32           state after draft token k
+ *   states_out  [B, K, H, P, N]   fp32 or NULL   state after draft token k
  *   y           [B, K, H, P]      dtype          outputs of the K tokens
- * Requires dstate % 4 == 0.
+ * Requires dstate % 4 == 0. With states_out == NULL only y is written: the flow
+ * that keeps one state (ssd_advance_state below) instead of all K.
  */
 ssd_status_t ssd_verify(const ssd_shape_t *shape, ssd_dtype_t dtype, const float *h0,
                         const void *x, const void *dt, const float *A, const void *Bm,
@@ -176,6 +177,42 @@ ssd_status_t ssd_verify(const ssd_shape_t *shape, ssd_dtype_t dtype, const float
 ssd_status_t ssd_select_state(const ssd_shape_t *shape, int64_t K, const float *h0,
                               const float *states_out, const int32_t *accepted, float *h_keep,
                               void *stream);
+
+/*
+ * The kept state without storing the intermediate ones. The distillation
+ * write-up ("推测解码") notes that keeping every intermediate state of a verify
+ * pass costs too much memory; the state at the accepted position is what is
+ * needed. Once the caller knows how many draft tokens of each batch row were
+ * accepted, this recomputes that state from h0:
+ *   h_keep[b] = state after the first accepted[b] tokens, starting from h0[b]
+ *             (accepted[b] == 0: a copy of h0[b])
+ * Same arguments and layouts as ssd_verify (shape->seqlen == K); `accepted` is a
+ * device int32 array [B]. The result is bit-identical to ssd_verify's
+ * states_out[b, accepted[b]-1] (the same fp32 operations in the same order). A row
+ * whose count is outside 0..K is filled with quiet NaN. h_keep may be h0 itself
+ * (the state advanced in place); no other overlap between them is allowed
+ * (SSD_ERR_INVALID_ARG). Requires dstate % 4 == 0 and K <= 64.
+ */
+ssd_status_t ssd_advance_state(const ssd_shape_t *shape, ssd_dtype_t dtype, const float *h0,
+                               const void *x, const void *dt, const float *A, const void *Bm,
+                               int64_t K, const int32_t *accepted, float *h_keep, void *stream);
+
+/*
+ * One generated token (the recurrent form, "The Recurrent Representation" of the
+ * visual guide): the state is updated in place,
+ *   state <- exp(dt * A_h) * state + dt * x B^T,   y = state C + D_h * x
+ * shape->seqlen must be 1.
+ *   state   [B, H, P, N]   fp32           read and written
+ *   x       [B, H, P]      dtype
+ *   dt      [B, H]         dtype
+ *   A, D    [H]            fp32 (D may be NULL = 0)
+ *   Bm, Cm  [B, G, N]      dtype
+ *   y       [B, H, P]      dtype
+ * Requires dstate % 4 == 0. Same arithmetic as ssd_verify with K = 1.
+ */
+ssd_status_t ssd_decode_step(const ssd_shape_t *shape, ssd_dtype_t dtype, float *state,
+                             const void *x, const void *dt, const float *A, const void *Bm,
+                             const void *Cm, const float *D, void *y, void *stream);
 
 #ifdef __cplusplus
 }

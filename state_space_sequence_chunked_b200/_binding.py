@@ -45,6 +45,8 @@ _SIGS = {
     "ssd_fwd": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 7 + [_i64, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "ssd_verify": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 7 + [_i64, _vp, _vp, _vp], ctypes.c_int),
     "ssd_select_state": ([ctypes.POINTER(ShapeT), _i64] + [_vp] * 5, ctypes.c_int),
+    "ssd_advance_state": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 5 + [_i64, _vp, _vp, _vp], ctypes.c_int),
+    "ssd_decode_step": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 9, ctypes.c_int),
 }
 
 
@@ -138,15 +140,18 @@ def ssd_fwd(x, dt, A, B, C, D=None, h0=None, *, chunk: int, y=None, h_final=None
     return y, h_final
 
 
-def ssd_verify(h0, x, dt, A, B, C, D=None, *, states_out=None, y=None, stream=None):
-    """y [B,K,H,P], states_out [B,K,H,P,N] = ssd_verify(h0 [B,H,P,N] f32, x [B,K,H,P], dt, A, B, C, D)."""
+def ssd_verify(h0, x, dt, A, B, C, D=None, *, states_out=None, y=None, return_states: bool = True,
+               stream=None):
+    """y [B,K,H,P], states_out [B,K,H,P,N] = ssd_verify(h0 [B,H,P,N] f32, x [B,K,H,P], dt, A, B, C, D).
+
+    return_states=False (and no states_out given) writes y only; states_out is then None."""
     dev = _dev(h0, x, dt, A, B, C, D, states_out, y)
     Bsz, K, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
     shape = ShapeT(Bsz, K, H, P, G, N)
     if y is None:
         y = torch.empty_like(x)
-    if states_out is None:
+    if states_out is None and return_states:
         states_out = torch.empty((Bsz, K, H, P, N), dtype=torch.float32, device=dev)
     st = lib().ssd_verify(ctypes.byref(shape), _dtype_code(x), _ptr(h0), _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
                           _ptr(C), _ptr(D), K, _ptr(states_out), _ptr(y), _stream(dev, stream))
@@ -167,3 +172,34 @@ def ssd_select_state(h0, states_out, accepted, *, h_keep=None, stream=None):
                                 _ptr(h_keep), _stream(dev, stream))
     _check(st, "ssd_select_state")
     return h_keep
+
+
+def ssd_advance_state(h0, x, dt, A, B, accepted, *, h_keep=None, stream=None):
+    """h_keep[b] = state after the first accepted[b] draft tokens from h0[b] (h_keep may be h0: in place)."""
+    dev = _dev(h0, x, dt, A, B, accepted, h_keep)
+    if accepted.dtype != torch.int32:
+        raise TypeError("accepted must be int32")
+    Bsz, K, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    shape = ShapeT(Bsz, K, H, P, G, N)
+    if h_keep is None:
+        h_keep = torch.empty_like(h0)
+    st = lib().ssd_advance_state(ctypes.byref(shape), _dtype_code(x), _ptr(h0), _ptr(x), _ptr(dt), _ptr(A),
+                                 _ptr(B), K, _ptr(accepted), _ptr(h_keep), _stream(dev, stream))
+    _check(st, "ssd_advance_state")
+    return h_keep
+
+
+def ssd_decode_step(state, x, dt, A, B, C, D=None, *, y=None, stream=None):
+    """One token in place: state [B,H,P,N] f32 <- exp(dt A) state + dt x B^T; returns y [B,H,P] = state C + D x.
+    x [B,H,P], dt [B,H], B/C [B,G,N]."""
+    dev = _dev(state, x, dt, A, B, C, D, y)
+    Bsz, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    shape = ShapeT(Bsz, 1, H, P, G, N)
+    if y is None:
+        y = torch.empty_like(x)
+    st = lib().ssd_decode_step(ctypes.byref(shape), _dtype_code(x), _ptr(state), _ptr(x), _ptr(dt), _ptr(A),
+                               _ptr(B), _ptr(C), _ptr(D), _ptr(y), _stream(dev, stream))
+    _check(st, "ssd_decode_step")
+    return y

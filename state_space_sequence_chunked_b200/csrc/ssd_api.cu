@@ -153,7 +153,7 @@ SSD_API ssd_status_t ssd_verify(const ssd_shape_t *shape, ssd_dtype_t dtype, con
     if (K < 1 || shape->seqlen != K) return SSD_ERR_INVALID_ARG;
     if (K > kMaxVerifyK || shape->dstate % 4 != 0) return SSD_ERR_UNSUPPORTED;
     if (shape->batch == 0) return SSD_OK;
-    if (!h0 || !x || !dt || !A || !Bm || !Cm || !states_out || !y) return SSD_ERR_INVALID_ARG;
+    if (!h0 || !x || !dt || !A || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;  // states_out optional
     const void *ptrs[] = {h0, x, dt, A, Bm, Cm, D, states_out, y};
     for (const void *q : ptrs)
         if (q && !aligned16(q)) return SSD_ERR_ALIGNMENT;
@@ -177,4 +177,44 @@ SSD_API ssd_status_t ssd_select_state(const ssd_shape_t *shape, int64_t K, const
     const int64_t per_row = shape->nheads * shape->headdim * shape->dstate;
     return from_cuda(select_launch(shape->batch, K, per_row, h0, states_out, accepted, h_keep,
                                    static_cast<cudaStream_t>(stream)));
+}
+
+SSD_API ssd_status_t ssd_advance_state(const ssd_shape_t *shape, ssd_dtype_t dtype, const float *h0,
+                                       const void *x, const void *dt, const float *A, const void *Bm,
+                                       int64_t K, const int32_t *accepted, float *h_keep, void *stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if ((st = check_dtype(dtype)) != SSD_OK) return st;
+    if (K < 1 || shape->seqlen != K) return SSD_ERR_INVALID_ARG;
+    if (K > kMaxVerifyK || shape->dstate % 4 != 0) return SSD_ERR_UNSUPPORTED;
+    if (shape->batch == 0) return SSD_OK;
+    if (!h0 || !x || !dt || !A || !Bm || !accepted || !h_keep) return SSD_ERR_INVALID_ARG;
+    const void *ptrs[] = {h0, x, dt, A, Bm, accepted, h_keep};
+    for (const void *q : ptrs)
+        if (!aligned16(q)) return SSD_ERR_ALIGNMENT;
+    // h_keep may be h0 itself (in place); any other overlap is not allowed.
+    const size_t state_bytes = (size_t)(shape->batch * shape->nheads * shape->headdim * shape->dstate) * sizeof(float);
+    const char *a0 = reinterpret_cast<const char *>(h0), *k0 = reinterpret_cast<const char *>(h_keep);
+    if (a0 != k0 && a0 < k0 + state_bytes && k0 < a0 + state_bytes) return SSD_ERR_INVALID_ARG;
+    VerifyProblem p{shape->batch, K, shape->nheads, shape->headdim, shape->ngroups, shape->dstate,
+                    dtype, h0, x, dt, Bm, nullptr, A, nullptr, nullptr, nullptr};
+    return from_cuda(advance_launch(p, accepted, h_keep, static_cast<cudaStream_t>(stream)));
+}
+
+SSD_API ssd_status_t ssd_decode_step(const ssd_shape_t *shape, ssd_dtype_t dtype, float *state,
+                                     const void *x, const void *dt, const float *A, const void *Bm,
+                                     const void *Cm, const float *D, void *y, void *stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if ((st = check_dtype(dtype)) != SSD_OK) return st;
+    if (shape->seqlen != 1) return SSD_ERR_INVALID_ARG;
+    if (shape->dstate % 4 != 0) return SSD_ERR_UNSUPPORTED;
+    if (shape->batch == 0) return SSD_OK;
+    if (!state || !x || !dt || !A || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;
+    const void *ptrs[] = {state, x, dt, A, Bm, Cm, D, y};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return SSD_ERR_ALIGNMENT;
+    VerifyProblem p{shape->batch, 1, shape->nheads, shape->headdim, shape->ngroups, shape->dstate,
+                    dtype, nullptr, x, dt, Bm, Cm, A, D, nullptr, y};
+    return from_cuda(decode_launch(p, state, static_cast<cudaStream_t>(stream)));
 }

@@ -43,6 +43,10 @@ cudaError_t tc_fwd(const FwdProblem &p, void *ws, cudaStream_t s);
 
 // ---- verify / select --------------------------------------------------------------
 cudaError_t verify_launch(const VerifyProblem &p, cudaStream_t s);
+// states_out may be NULL (outputs only). k_advance: state after accepted[b] tokens.
+// k_decode: one token, state updated in place (p.h0 and p.states_out unused).
+cudaError_t advance_launch(const VerifyProblem &p, const int32_t *accepted, float *h_keep, cudaStream_t s);
+cudaError_t decode_launch(const VerifyProblem &p, float *state, cudaStream_t s);
 cudaError_t select_launch(int64_t B, int64_t K, int64_t per_row, const float *h0,
                           const float *states_out, const int32_t *accepted, float *h_keep,
                           cudaStream_t s);

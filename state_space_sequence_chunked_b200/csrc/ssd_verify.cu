@@ -6,6 +6,15 @@
 // is the one at the position where the check stops). With K small the chunked
 // form has nothing to amortise, so each state row is advanced token by token in
 // registers; the cost is the K state writes, a pure HBM stream.
+//
+// The same write-up notes that storing every intermediate state is what a
+// hardware-aware verify should avoid. Two kernels serve that flow without states_out:
+// verify with states_out = NULL writes only y, and k_advance recomputes, once the
+// accepted counts are known, the state after accepted[b] tokens straight from h0
+// (K small steps per state row in registers: one read of h0 and one write of the
+// kept state). It applies the same fp32 operations in the same order as k_verify,
+// so its result is bit-identical to the verify state it replaces. k_decode is the
+// one-token step of generation, updating the state in place.
 #include "ssd_internal.cuh"
 
 namespace ssd {
@@ -64,7 +73,8 @@ __global__ void __launch_bounds__(kVThreads)
             const float dx = dts[k] * xk;
             const float4 *bk = reinterpret_cast<const float4 *>(bsm + k * N);
             const float4 *ck = reinterpret_cast<const float4 *>(csm + k * N);
-            float4 *dst = reinterpret_cast<float4 *>(states_out + ((((int64_t)b * K + k) * H + h) * P + p) * N);
+            float4 *dst = states_out ? reinterpret_cast<float4 *>(states_out + ((((int64_t)b * K + k) * H + h) * P + p) * N)
+                                     : nullptr;
             float part = 0.f;
 #pragma unroll
             for (int j = 0; j < kMaxVec; ++j) {
@@ -79,13 +89,145 @@ __global__ void __launch_bounds__(kVThreads)
                     part = fmaf(s[j].y, cc.y, part);
                     part = fmaf(s[j].z, cc.z, part);
                     part = fmaf(s[j].w, cc.w, part);
-                    __stcs(dst + v, s[j]);
+                    if (states_out) __stcs(dst + v, s[j]);
                 }
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
             if (lane == 0) store_as(y + (((int64_t)b * K + k) * H + h) * P + p, part + Dh * xk);
         }
+    }
+}
+
+// grid (H, B). The state after accepted[b] draft tokens, from h0: the update of
+// k_verify without the outputs. Shared memory: B (K x N), x (K x P), dt, decay (K).
+// A row whose count is outside 0..K is filled with quiet NaN.
+template <typename T>
+__global__ void __launch_bounds__(kVThreads)
+    k_advance(const float *__restrict__ h0, const T *__restrict__ x, const T *__restrict__ dt,
+              const float *__restrict__ A, const T *__restrict__ Bm, const int32_t *__restrict__ accepted,
+              int K, int H, int P, int G, int N, float *__restrict__ h_keep) {
+    extern __shared__ float sm[];
+    const int h = blockIdx.x, b = blockIdx.y, g = h / (H / G);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nv = N / 4;
+    const int a = accepted[b];
+    if (a < 0 || a > K) {
+        const float qn = __int_as_float(0x7fc00000);
+        float4 *dst = reinterpret_cast<float4 *>(h_keep + ((int64_t)b * H + h) * P * N);
+        for (int i = tid; i < P * nv; i += blockDim.x) dst[i] = make_float4(qn, qn, qn, qn);
+        return;
+    }
+    float *bsm = sm;            // [a][N]
+    float *xsm = bsm + a * N;   // [a][P]
+    float *dts = xsm + a * P;   // [a]
+    float *dec = dts + a;       // [a]
+    for (int i = tid; i < a * N; i += blockDim.x) {
+        const int k = i / N, n = i % N;
+        bsm[i] = to_f32(Bm[(((int64_t)b * K + k) * G + g) * N + n]);
+    }
+    for (int i = tid; i < a * P; i += blockDim.x) {
+        const int k = i / P, q = i % P;
+        xsm[i] = to_f32(x[(((int64_t)b * K + k) * H + h) * P + q]);
+    }
+    for (int k = tid; k < a; k += blockDim.x) {
+        const float d = to_f32(dt[((int64_t)b * K + k) * H + h]);
+        dts[k] = d;
+        dec[k] = expf(d * A[h]);
+    }
+    __syncthreads();
+    for (int p = warp; p < P; p += kVThreads / 32) {
+        const float4 *src = reinterpret_cast<const float4 *>(h0 + (((int64_t)b * H + h) * P + p) * N);
+        float4 *dst = reinterpret_cast<float4 *>(h_keep + (((int64_t)b * H + h) * P + p) * N);
+        float4 s[kMaxVec];
+#pragma unroll
+        for (int j = 0; j < kMaxVec; ++j) {
+            const int v = lane + 32 * j;
+            s[j] = v < nv ? src[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        for (int k = 0; k < a; ++k) {
+            const float dk = dec[k];
+            const float dx = dts[k] * xsm[k * P + p];
+            const float4 *bk = reinterpret_cast<const float4 *>(bsm + k * N);
+#pragma unroll
+            for (int j = 0; j < kMaxVec; ++j) {
+                const int v = lane + 32 * j;
+                if (v < nv) {
+                    const float4 bb = bk[v];
+                    s[j].x = fmaf(dk, s[j].x, dx * bb.x);
+                    s[j].y = fmaf(dk, s[j].y, dx * bb.y);
+                    s[j].z = fmaf(dk, s[j].z, dx * bb.z);
+                    s[j].w = fmaf(dk, s[j].w, dx * bb.w);
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxVec; ++j) {
+            const int v = lane + 32 * j;
+            if (v < nv) __stcs(dst + v, s[j]);
+        }
+    }
+}
+
+// grid (H, B). One token of generation, in place: state <- exp(dt A) state + dt x B^T,
+// y = state C + D x. Each state row is read whole into registers before it is
+// written back, and only its own warp touches it, so reading and writing the same
+// buffer is safe (which is why `state` carries no __restrict__).
+template <typename T>
+__global__ void __launch_bounds__(kVThreads)
+    k_decode(float *state, const T *__restrict__ x, const T *__restrict__ dt, const float *__restrict__ A,
+             const T *__restrict__ Bm, const T *__restrict__ Cm, const float *__restrict__ D, int H, int P,
+             int G, int N, T *__restrict__ y) {
+    extern __shared__ float sm[];
+    float *bsm = sm;        // [N]
+    float *csm = bsm + N;   // [N]
+    const int h = blockIdx.x, b = blockIdx.y, g = h / (H / G);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int n = tid; n < N; n += blockDim.x) {
+        const int64_t off = ((int64_t)b * G + g) * N + n;
+        bsm[n] = to_f32(Bm[off]);
+        csm[n] = to_f32(Cm[off]);
+    }
+    __syncthreads();
+    const float d = to_f32(dt[(int64_t)b * H + h]);
+    const float dk = expf(d * A[h]);
+    const float Dh = D ? D[h] : 0.f;
+    const int nv = N / 4;
+    for (int p = warp; p < P; p += kVThreads / 32) {
+        float4 *row = reinterpret_cast<float4 *>(state + (((int64_t)b * H + h) * P + p) * N);
+        const float xk = to_f32(x[((int64_t)b * H + h) * P + p]);
+        const float dx = d * xk;
+        float4 s[kMaxVec];
+#pragma unroll
+        for (int j = 0; j < kMaxVec; ++j) {
+            const int v = lane + 32 * j;
+            s[j] = v < nv ? row[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float part = 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxVec; ++j) {
+            const int v = lane + 32 * j;
+            if (v < nv) {
+                const float4 bb = reinterpret_cast<const float4 *>(bsm)[v];
+                const float4 cc = reinterpret_cast<const float4 *>(csm)[v];
+                s[j].x = fmaf(dk, s[j].x, dx * bb.x);
+                s[j].y = fmaf(dk, s[j].y, dx * bb.y);
+                s[j].z = fmaf(dk, s[j].z, dx * bb.z);
+                s[j].w = fmaf(dk, s[j].w, dx * bb.w);
+                part = fmaf(s[j].x, cc.x, part);
+                part = fmaf(s[j].y, cc.y, part);
+                part = fmaf(s[j].z, cc.z, part);
+                part = fmaf(s[j].w, cc.w, part);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxVec; ++j) {
+            const int v = lane + 32 * j;
+            if (v < nv) row[v] = s[j];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (lane == 0) store_as(y + ((int64_t)b * H + h) * P + p, part + Dh * xk);
     }
 }
 
@@ -128,6 +270,42 @@ cudaError_t verify_launch(const VerifyProblem &p, cudaStream_t s) {
         k_verify<bf><<<grid, kVThreads, smem, s>>>(p.h0, (const bf *)p.x, (const bf *)p.dt, p.A,
                                                    (const bf *)p.Bm, (const bf *)p.Cm, p.D, K, H, P, G, N,
                                                    p.states_out, (bf *)p.y);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t advance_launch(const VerifyProblem &p, const int32_t *accepted, float *h_keep, cudaStream_t s) {
+    const int K = (int)p.K, H = (int)p.H, P = (int)p.P, G = (int)p.G, N = (int)p.N;
+    const size_t smem = (size_t)(K * N + K * P + 2 * K) * sizeof(float);  // room for a = K
+    dim3 grid(H, (unsigned)p.B);
+    cudaError_t e;
+    if (p.dtype == SSD_F32) {
+        if ((e = cudaFuncSetAttribute(k_advance<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+            return e;
+        k_advance<float><<<grid, kVThreads, smem, s>>>(p.h0, (const float *)p.x, (const float *)p.dt, p.A,
+                                                       (const float *)p.Bm, accepted, K, H, P, G, N, h_keep);
+    } else {
+        using bf = __nv_bfloat16;
+        if ((e = cudaFuncSetAttribute(k_advance<bf>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+            return e;
+        k_advance<bf><<<grid, kVThreads, smem, s>>>(p.h0, (const bf *)p.x, (const bf *)p.dt, p.A, (const bf *)p.Bm,
+                                                    accepted, K, H, P, G, N, h_keep);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t decode_launch(const VerifyProblem &p, float *state, cudaStream_t s) {
+    const int H = (int)p.H, P = (int)p.P, G = (int)p.G, N = (int)p.N;
+    const size_t smem = (size_t)(2 * N) * sizeof(float);
+    dim3 grid(H, (unsigned)p.B);
+    if (p.dtype == SSD_F32) {
+        k_decode<float><<<grid, kVThreads, smem, s>>>(state, (const float *)p.x, (const float *)p.dt, p.A,
+                                                      (const float *)p.Bm, (const float *)p.Cm, p.D, H, P, G, N,
+                                                      (float *)p.y);
+    } else {
+        using bf = __nv_bfloat16;
+        k_decode<bf><<<grid, kVThreads, smem, s>>>(state, (const bf *)p.x, (const bf *)p.dt, p.A, (const bf *)p.Bm,
+                                                   (const bf *)p.Cm, p.D, H, P, G, N, (bf *)p.y);
     }
     return cudaGetLastError();
 }

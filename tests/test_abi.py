@@ -32,7 +32,8 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for n in ("ssd_fwd", "ssd_verify", "ssd_select_state", "ssd_fwd_workspace_bytes", "ssd_strerror"):
+    for n in ("ssd_fwd", "ssd_verify", "ssd_select_state", "ssd_fwd_workspace_bytes", "ssd_strerror",
+              "ssd_advance_state", "ssd_decode_step"):
         assert n in names
 
 
@@ -127,6 +128,33 @@ def test_verify_and_select_reject_before_launch(lib):
     assert sel(acc=None) == 1
     assert sel(acc=0x4004) == 3
     assert sel(shape=B.ShapeT(2, 8, 4, 16, 2, 6)) == 2
+
+
+def test_advance_and_decode_reject_before_launch(lib):
+    s = B.ShapeT(2, 8, 4, 16, 2, 16)
+    vp = lambda a: ctypes.c_void_p(a) if a else None
+
+    def adv(shape=s, K=8, h0=0x1000, acc=0x4000, keep=0x100000, x=0x2000):
+        return lib.ssd_advance_state(ctypes.byref(shape), 1, vp(h0), vp(x), vp(0x3000), vp(0x3100), vp(0x3200), K,
+                                     vp(acc), vp(keep), None)
+
+    assert adv(K=7) == 1                                   # seqlen != K
+    assert adv(K=65, shape=B.ShapeT(2, 65, 4, 16, 2, 16)) == 2
+    assert adv(shape=B.ShapeT(2, 8, 4, 16, 2, 18)) == 2     # dstate % 4
+    assert adv(acc=None) == 1
+    assert adv(x=0x2008) == 3
+    assert adv(keep=0x1010) == 1                           # overlaps h0 without being it
+    assert adv(shape=B.ShapeT(0, 8, 4, 16, 2, 16), h0=None, acc=None, keep=None) == 0   # empty batch
+
+    def dec(shape=B.ShapeT(2, 1, 4, 16, 2, 16), state=0x1000, y=0x5000, D=None):
+        return lib.ssd_decode_step(ctypes.byref(shape), 1, vp(state), vp(0x2000), vp(0x3000), vp(0x3100),
+                                   vp(0x3200), vp(0x3300), vp(D), vp(y), None)
+
+    assert dec(shape=B.ShapeT(2, 2, 4, 16, 2, 16)) == 1   # seqlen must be 1
+    assert dec(shape=B.ShapeT(2, 1, 4, 16, 2, 6)) == 2
+    assert dec(state=None) == 1
+    assert dec(y=0x5002) == 3
+    assert dec(D=0x6004) == 3
 
 
 def test_binding_requires_cuda_tensors():

@@ -81,3 +81,65 @@ def test_select_every_index_and_out_of_range(cuda_device):
         assert torch.equal(kept[b].view(torch.int32), want.view(torch.int32))
     assert torch.isnan(kept[9]).all() and torch.isnan(kept[10]).all()
     assert torch.equal(kept[11], so[11, 7])
+
+
+def test_verify_outputs_only_and_advance_state_full_workload(cuda_device):
+    """The flow that keeps one state instead of K (full verify workload): verify with no
+    states_out gives the same y bit for bit, and the state recomputed for the drawn accepted
+    counts equals ssd_select_state over the stored states bit for bit, also in place."""
+    d = draw("verify_k8")
+    g, y, so = run_verify(d, cuda_device)
+    y2, none = ssd.ssd_verify(g["h0"], g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], return_states=False)
+    acc = torch.from_numpy(d["accepted"]).to(cuda_device)
+    kept = ssd.ssd_select_state(g["h0"], so, acc)
+    adv = ssd.ssd_advance_state(g["h0"], g["x"], g["dt"], g["A"], g["B"], acc)
+    inplace = g["h0"].clone()
+    ret = ssd.ssd_advance_state(inplace, g["x"], g["dt"], g["A"], g["B"], acc, h_keep=inplace)
+    torch.cuda.synchronize()
+    assert none is None and ret is inplace
+    assert torch.equal(y2.view(torch.int16), y.view(torch.int16))
+    assert torch.equal(adv.view(torch.int32), kept.view(torch.int32))
+    assert torch.equal(inplace.view(torch.int32), kept.view(torch.int32))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_advance_state_every_count(cuda_device, dtype):
+    """Every accepted count 0..K on its own row, plus two out-of-range rows (NaN), against the
+    stored verify states bit for bit and against the oracle's state after that many tokens."""
+    K = 6
+    wl = dataclasses.replace(inputs.WORKLOADS["verify_k8"], batch=K + 3, seqlen=K, nheads=4, headdim=32,
+                             ngroups=2, dstate=64, dtype=dtype, seed=77)
+    d = inputs.draw(wl)
+    g, y, so = run_verify(d, cuda_device)
+    acc_list = list(range(K + 1)) + [-1, K + 1]
+    acc = torch.tensor(acc_list, dtype=torch.int32, device=cuda_device)
+    adv = ssd.ssd_advance_state(g["h0"], g["x"], g["dt"], g["A"], g["B"], acc)
+    torch.cuda.synchronize()
+    _, sr = oracle_rows(d, (0, K + 3))
+    h0r = d["h0"].value
+    for b, a in enumerate(acc_list):
+        if a < 0 or a > K:
+            assert torch.isnan(adv[b]).all()
+            continue
+        want = g["h0"][b] if a == 0 else so[b, a - 1]
+        assert torch.equal(adv[b].view(torch.int32), want.view(torch.int32)), b
+        ref = h0r[b] if a == 0 else sr[b, a - 1]
+        assert rel_err(to_np(adv[b]), ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype,H,P,G,N", [("bf16", 32, 128, 8, 128), ("f32", 4, 16, 2, 16), ("bf16", 3, 8, 1, 256)])
+def test_decode_step(cuda_device, dtype, H, P, G, N):
+    """One token in place: equals ssd_verify with K = 1 bit for bit (y and state), and the oracle."""
+    wl = dataclasses.replace(inputs.WORKLOADS["verify_k8"], batch=5, seqlen=1, nheads=H, headdim=P, ngroups=G,
+                             dstate=N, dtype=dtype, seed=91)
+    d = inputs.draw(wl)
+    g, y, so = run_verify(d, cuda_device)
+    state = g["h0"].clone()
+    yd = ssd.ssd_decode_step(state, g["x"][:, 0].contiguous(), g["dt"][:, 0].contiguous(), g["A"],
+                             g["B"][:, 0].contiguous(), g["C"][:, 0].contiguous(), g["D"])
+    torch.cuda.synchronize()
+    assert torch.equal(state.view(torch.int32), so[:, 0].view(torch.int32))
+    assert torch.equal(yd.float(), y[:, 0].float())
+    yr, sr = oracle_rows(d, (0, 5))
+    assert rel_err(to_np(yd), yr[:, 0]) <= TOL[dtype]
+    assert rel_err(to_np(state), sr[:, 0]) <= TOL[dtype]
