@@ -214,6 +214,60 @@ ssd_status_t ssd_decode_step(const ssd_shape_t *shape, ssd_dtype_t dtype, float 
                              const void *x, const void *dt, const float *A, const void *Bm,
                              const void *Cm, const float *D, void *y, void *stream);
 
+/*
+ * Context (sequence) parallelism: a long sequence split into contiguous segments,
+ * one per rank (the SSD write-up, "序列并行", built on the state passing of
+ * "SSD 算法：分块和状态传递"). Each rank runs ssd_fwd on its segment (rank 0 with
+ * the true h0, the others from zeros), which gives its local outputs y and local
+ * end state S_r; then:
+ *   1. ssd_cp_decay:   the segment's decay sums (per 128-token block, and the total
+ *                      Lambda_r = sum over the segment of dt_t * A_h);
+ *   2. the caller all-gathers S_r [B,H,P,N] and Lambda_r [B,H] over the ranks, in
+ *      rank order (one collective; ncclAllGather through torch.distributed);
+ *   3. ssd_cp_combine: the state entering this segment, the exclusive scan
+ *        S_in(0) = 0,  S_in(q+1) = exp(Lambda_q) S_in(q) + S_q,
+ *      and the segment's true end state exp(Lambda_r) S_in(r) + S_r;
+ *   4. ssd_cp_correct: y_t += exp(sum_{s<=t in segment} dt_s A_h) C_t S_in(r)^T, the
+ *      state-to-output step for the incoming state (a no-op for rank 0).
+ * Shapes below are those of the rank's segment (shape->seqlen = its length).
+ */
+#define SSD_CP_BLOCK 128 /* tokens per decay block: block_decay has ceil(seqlen/128) per (b, h) */
+
+/*
+ *   dt           [B, L, H]             dtype
+ *   A            [H]                   fp32
+ *   block_decay  [B, H, ceil(L/128)]   fp32   sum of dt*A over each 128-token block
+ *   total        [B, H]                fp32   Lambda = the block sums added in order
+ * L == 0 writes total = 0 (dt and block_decay may then be NULL).
+ */
+ssd_status_t ssd_cp_decay(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *dt, const float *A,
+                          float *block_decay, float *total, void *stream);
+
+/*
+ *   states   [R, B, H, P, N]   fp32   every rank's local end state, in rank order
+ *   totals   [R, B, H]         fp32   every rank's Lambda, in rank order
+ *   s_in     [B, H, P, N]      fp32   out: the state entering segment `rank`
+ *   h_final  [B, H, P, N]      fp32 or NULL   out: the true end state of segment `rank`
+ *                                     (for the last rank: the whole sequence's h_final)
+ * R = nranks >= 1, 0 <= rank < R. shape->seqlen and shape->ngroups are ignored.
+ * Requires headdim * dstate % 4 == 0. h_final must not overlap states.
+ */
+ssd_status_t ssd_cp_combine(const ssd_shape_t *shape, int64_t nranks, int64_t rank, const float *states,
+                            const float *totals, float *s_in, float *h_final, void *stream);
+
+/*
+ *   dt, Cm        as in ssd_fwd, for the segment
+ *   A             [H] fp32
+ *   block_decay   [B, H, ceil(L/128)] from ssd_cp_decay on the same segment
+ *   s_in          [B, H, P, N] fp32 from ssd_cp_combine
+ *   y             [B, L, H, P] dtype, read and written (y += the incoming state's term)
+ * bf16 inputs with headdim % 64 == 0 and dstate % 16 == 0 run on tensor cores (S_in
+ * rounded to bf16, fp32 accumulation); other shapes and fp32 inputs in fp32 on CUDA cores.
+ */
+ssd_status_t ssd_cp_correct(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *dt, const float *A,
+                            const void *Cm, const float *block_decay, const float *s_in, void *y,
+                            void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -47,7 +47,12 @@ _SIGS = {
     "ssd_select_state": ([ctypes.POINTER(ShapeT), _i64] + [_vp] * 5, ctypes.c_int),
     "ssd_advance_state": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 5 + [_i64, _vp, _vp, _vp], ctypes.c_int),
     "ssd_decode_step": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 9, ctypes.c_int),
+    "ssd_cp_decay": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 5, ctypes.c_int),
+    "ssd_cp_combine": ([ctypes.POINTER(ShapeT), _i64, _i64] + [_vp] * 5, ctypes.c_int),
+    "ssd_cp_correct": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 7, ctypes.c_int),
 }
+
+CP_BLOCK = 128  # SSD_CP_BLOCK: tokens per decay block
 
 
 def lib():
@@ -202,4 +207,48 @@ def ssd_decode_step(state, x, dt, A, B, C, D=None, *, y=None, stream=None):
     st = lib().ssd_decode_step(ctypes.byref(shape), _dtype_code(x), _ptr(state), _ptr(x), _ptr(dt), _ptr(A),
                                _ptr(B), _ptr(C), _ptr(D), _ptr(y), _stream(dev, stream))
     _check(st, "ssd_decode_step")
+    return y
+
+
+def ssd_cp_decay(dt, A, *, block_decay=None, total=None, stream=None):
+    """block_decay [B,H,ceil(L/128)], total [B,H] = sums of dt*A over a segment's blocks and over the segment."""
+    dev = _dev(dt, A, block_decay, total)
+    Bsz, L, H = dt.shape
+    nblk = (L + CP_BLOCK - 1) // CP_BLOCK
+    if block_decay is None:
+        block_decay = torch.empty((Bsz, H, max(nblk, 1)), dtype=torch.float32, device=dev)
+    if total is None:
+        total = torch.empty((Bsz, H), dtype=torch.float32, device=dev)
+    shape = ShapeT(Bsz, L, H, 1, 1, 1)
+    st = lib().ssd_cp_decay(ctypes.byref(shape), _dtype_code(dt), _ptr(dt), _ptr(A), _ptr(block_decay), _ptr(total),
+                            _stream(dev, stream))
+    _check(st, "ssd_cp_decay")
+    return block_decay, total
+
+
+def ssd_cp_combine(states, totals, rank, *, s_in=None, h_final=None, want_final=True, stream=None):
+    """s_in (state entering segment `rank`), h_final (its true end state) from the gathered
+    states [R,B,H,P,N] and totals [R,B,H]."""
+    dev = _dev(states, totals, s_in, h_final)
+    R, Bsz, H, P, N = states.shape
+    if s_in is None:
+        s_in = torch.empty((Bsz, H, P, N), dtype=torch.float32, device=dev)
+    if h_final is None and want_final:
+        h_final = torch.empty((Bsz, H, P, N), dtype=torch.float32, device=dev)
+    shape = ShapeT(Bsz, 0, H, P, 1, N)
+    st = lib().ssd_cp_combine(ctypes.byref(shape), R, rank, _ptr(states), _ptr(totals), _ptr(s_in), _ptr(h_final),
+                              _stream(dev, stream))
+    _check(st, "ssd_cp_combine")
+    return s_in, h_final
+
+
+def ssd_cp_correct(dt, A, C, block_decay, s_in, y, *, stream=None):
+    """y += exp(cumulative dt*A from the segment start) * C S_in^T, in place; returns y."""
+    dev = _dev(dt, A, C, block_decay, s_in, y)
+    Bsz, L, H, P = y.shape
+    G, N = C.shape[2], C.shape[3]
+    shape = ShapeT(Bsz, L, H, P, G, N)
+    st = lib().ssd_cp_correct(ctypes.byref(shape), _dtype_code(y), _ptr(dt), _ptr(A), _ptr(C), _ptr(block_decay),
+                              _ptr(s_in), _ptr(y), _stream(dev, stream))
+    _check(st, "ssd_cp_correct")
     return y

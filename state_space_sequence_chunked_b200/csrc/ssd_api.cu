@@ -218,3 +218,56 @@ SSD_API ssd_status_t ssd_decode_step(const ssd_shape_t *shape, ssd_dtype_t dtype
                     dtype, nullptr, x, dt, Bm, Cm, A, D, nullptr, y};
     return from_cuda(decode_launch(p, state, static_cast<cudaStream_t>(stream)));
 }
+
+// ---- context parallelism ------------------------------------------------------------
+
+namespace {
+ssd::CpProblem make_cp(const ssd_shape_t *s, ssd_dtype_t dtype) {
+    return ssd::CpProblem{s->batch, s->seqlen, s->nheads, s->headdim, s->ngroups, s->dstate, dtype};
+}
+}  // namespace
+
+SSD_API ssd_status_t ssd_cp_decay(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *dt, const float *A,
+                                  float *block_decay, float *total, void *stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if ((st = check_dtype(dtype)) != SSD_OK) return st;
+    if (shape->batch == 0) return SSD_OK;
+    if (!A || !total || (shape->seqlen > 0 && (!dt || !block_decay))) return SSD_ERR_INVALID_ARG;
+    const void *ptrs[] = {dt, A, block_decay, total};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return SSD_ERR_ALIGNMENT;
+    return from_cuda(cp_block_decay_launch(make_cp(shape, dtype), dt, A, block_decay, total,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+SSD_API ssd_status_t ssd_cp_combine(const ssd_shape_t *shape, int64_t nranks, int64_t rank, const float *states,
+                                    const float *totals, float *s_in, float *h_final, void *stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (nranks < 1 || rank < 0 || rank >= nranks) return SSD_ERR_INVALID_ARG;
+    if (nranks > 65536) return SSD_ERR_UNSUPPORTED;
+    if ((shape->headdim * shape->dstate) % 4 != 0) return SSD_ERR_UNSUPPORTED;
+    if (shape->batch == 0) return SSD_OK;
+    if (!states || !totals || !s_in) return SSD_ERR_INVALID_ARG;
+    const void *ptrs[] = {states, totals, s_in, h_final};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return SSD_ERR_ALIGNMENT;
+    return from_cuda(cp_combine_launch(make_cp(shape, SSD_F32), (int)nranks, (int)rank, states, totals, s_in,
+                                       h_final, static_cast<cudaStream_t>(stream)));
+}
+
+SSD_API ssd_status_t ssd_cp_correct(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *dt, const float *A,
+                                    const void *Cm, const float *block_decay, const float *s_in, void *y,
+                                    void *stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if ((st = check_dtype(dtype)) != SSD_OK) return st;
+    if (shape->batch == 0 || shape->seqlen == 0) return SSD_OK;
+    if (!dt || !A || !Cm || !block_decay || !s_in || !y) return SSD_ERR_INVALID_ARG;
+    const void *ptrs[] = {dt, A, Cm, block_decay, s_in, y};
+    for (const void *q : ptrs)
+        if (!aligned16(q)) return SSD_ERR_ALIGNMENT;
+    return from_cuda(cp_correct_launch(make_cp(shape, dtype), dt, A, Cm, block_decay, s_in, y,
+                                       static_cast<cudaStream_t>(stream)));
+}

@@ -29,6 +29,12 @@ struct VerifyProblem {
     void *y;
 };
 
+// A sequence segment for the context-parallel steps (ssd_cp_*).
+struct CpProblem {
+    int64_t B, L, H, P, G, N;
+    ssd_dtype_t dtype;
+};
+
 constexpr size_t kWsAlign = 256;
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -50,6 +56,16 @@ cudaError_t decode_launch(const VerifyProblem &p, float *state, cudaStream_t s);
 cudaError_t select_launch(int64_t B, int64_t K, int64_t per_row, const float *h0,
                           const float *states_out, const int32_t *accepted, float *h_keep,
                           cudaStream_t s);
+
+// ---- context parallelism: decay sums, the exchange scan, the state-to-output correction
+int cp_nblk(int64_t L);
+cudaError_t cp_block_decay_launch(const CpProblem &p, const void *dt, const float *A, float *bsum, float *total,
+                                  cudaStream_t s);
+cudaError_t cp_combine_launch(const CpProblem &p, int R, int rank, const float *states, const float *totals,
+                              float *s_in, float *h_final, cudaStream_t s);
+bool cp_correct_uses_mma(const CpProblem &p);
+cudaError_t cp_correct_launch(const CpProblem &p, const void *dt, const float *A, const void *Cm, const float *bsum,
+                              const float *s_in, void *y, cudaStream_t s);
 
 // ---- element access ---------------------------------------------------------------
 __device__ __forceinline__ float to_f32(float v) { return v; }
