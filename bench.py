@@ -338,6 +338,101 @@ def verify_main(args, wl):
     return 0
 
 
+def aux_main(args):
+    """Per-kernel timings of the kernels beside the forward, each against the HBM roofline
+    (all of them are bandwidth-bound): the two verify flows on the spec-decode workload
+    (all K states stored + select, or outputs only + recomputing the kept state), the
+    one-token decode step at the same shape, and the three context-parallel steps for one
+    rank's eighth of the long-context sequence (B1 L8192 of L65536, H80 P64 N256). One JSON
+    line per kernel; inputs resident in HBM; CUDA events around `--steps` launches."""
+    import torch
+
+    from state_space_sequence_chunked_b200 import _binding as ssd
+    from state_space_sequence_chunked_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    hbm, _, src = peaks()
+    steps = max(args.steps, 1)
+
+    def timed(fn):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    def emit(kernel, workload, ms, alg_bytes, launches, **extra):
+        gbs = alg_bytes / (ms * 1e-3) / 1e9
+        print(json.dumps({"kernel": kernel, "workload": workload, "ms": ms, "alg_bytes": alg_bytes,
+                          "launches_per_call": launches, "achieved_gbs": gbs, "peak_gbs": hbm,
+                          "peak_source": src, "frac": gbs / hbm, "steps": steps, **extra}), flush=True)
+
+    # spec-decode verify workload: B64 K8 H32 P128 N128 G8, bf16 inputs, fp32 states
+    wl = inputs.WORKLOADS["verify_k8"]
+    d = inputs.draw(wl)
+    g = {k: d[k].torch(dev) for k in ("x", "dt", "A", "B", "C", "D", "h0")}
+    acc = torch.from_numpy(d["accepted"]).to(dev)
+    Bsz, K, H, P, N, G = wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.dstate, wl.ngroups
+    state = Bsz * H * P * N * 4
+    x_b, dt_b, bc_b = Bsz * K * H * P * 2, Bsz * K * H * 2, Bsz * K * G * N * 2  # x (= y), dt, B (= C)
+    small = 2 * x_b + dt_b + 2 * bc_b
+    so = torch.empty(Bsz, K, H, P, N, device=dev)
+    y = torch.empty_like(g["x"])
+    keep = torch.empty(Bsz, H, P, N, device=dev)
+    ms = timed(lambda: ssd.ssd_verify(g["h0"], g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], states_out=so, y=y,
+                                      stream=stream))
+    emit("k_verify (all K states)", wl.name, ms, state * (1 + K) + small, 1)
+    ms = timed(lambda: ssd.ssd_select_state(g["h0"], so, acc, h_keep=keep, stream=stream))
+    emit("k_select", wl.name, ms, 2 * state, 1)
+    ms = timed(lambda: ssd.ssd_verify(g["h0"], g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], y=y,
+                                      return_states=False, stream=stream))
+    emit("k_verify (outputs only)", wl.name, ms, state + small, 1)
+    ms = timed(lambda: ssd.ssd_advance_state(g["h0"], g["x"], g["dt"], g["A"], g["B"], acc, h_keep=keep,
+                                             stream=stream))
+    emit("k_advance", wl.name, ms, 2 * state + x_b + dt_b + bc_b, 1)
+    st = g["h0"].clone()
+    x1, dt1 = g["x"][:, 0].contiguous(), g["dt"][:, 0].contiguous()
+    B1, C1 = g["B"][:, 0].contiguous(), g["C"][:, 0].contiguous()
+    y1 = torch.empty_like(x1)
+    ms = timed(lambda: ssd.ssd_decode_step(st, x1, dt1, g["A"], B1, C1, g["D"], y=y1, stream=stream))
+    emit("k_decode (one token, in place)", "verify_k8 shape, K=1", ms, 2 * state + small // K, 1)  # small/K: one token
+    del so
+
+    # context parallelism: one of 8 segments of the long-context workload
+    wl = inputs.WORKLOADS["long_n256"]
+    R, Ls = 8, wl.seqlen // 8
+    d = inputs.draw(wl, seqlen=Ls)
+    g = {k: d[k].torch(dev) for k in ("x", "dt", "A", "B", "C", "D")}
+    Bsz, H, P, N, G = wl.batch, wl.nheads, wl.headdim, wl.dstate, wl.ngroups
+    nblk = (Ls + 127) // 128
+    bd = torch.empty(Bsz, H, nblk, device=dev)
+    tot = torch.empty(Bsz, H, device=dev)
+    ms = timed(lambda: ssd.ssd_cp_decay(g["dt"], g["A"], block_decay=bd, total=tot, stream=stream))
+    emit("k_block_decay + k_total_decay", f"long_n256 segment 1/{R}", ms, Bsz * Ls * H * 2 + Bsz * H * (nblk + 1) * 4,
+         2)
+    states = torch.randn(R, Bsz, H, P, N, device=dev) * 0.1
+    totals = -torch.rand(R, Bsz, H, device=dev)
+    s_in = torch.empty(Bsz, H, P, N, device=dev)
+    hf = torch.empty(Bsz, H, P, N, device=dev)
+    ms = timed(lambda: ssd.ssd_cp_combine(states, totals, R - 1, s_in=s_in, h_final=hf, stream=stream))
+    emit("k_combine (last of 8 ranks)", f"long_n256 B1 H80 P64 N256, R={R}", ms,
+         (R + 2) * Bsz * H * P * N * 4 + R * Bsz * H * 4, 1)
+    yseg = torch.zeros(Bsz, Ls, H, P, dtype=torch.bfloat16, device=dev)
+    ms = timed(lambda: ssd.ssd_cp_correct(g["dt"], g["A"], g["C"], bd, s_in, yseg, stream=stream))
+    flops = 2.0 * Bsz * Ls * H * P * N
+    emit("k_correct_mma", f"long_n256 segment 1/{R}", ms,
+         2 * Bsz * Ls * H * P * 2 + Bsz * Ls * G * N * 2 + Bsz * Ls * H * 2 + Bsz * H * P * N * 4, 1,
+         flops=flops, tflops=flops / (ms * 1e-3) / 1e12)
+    return 0
+
+
 # ---------------------------------------------------------------------------------------
 
 def main():
@@ -349,7 +444,11 @@ def main():
     ap.add_argument("--workload", default="mamba2_2p7b")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--aux", action="store_true",
+                    help="time the verify/decode and context-parallel kernels instead (1 GPU, one line per kernel)")
     args = ap.parse_args()
+    if args.aux:
+        return aux_main(args)
 
     from state_space_sequence_chunked_b200 import inputs
 

@@ -126,15 +126,25 @@ __global__ void __launch_bounds__(256)
     float *cum = reinterpret_cast<float *>(st + 64 * ld);               // [128]
     const int64_t t0 = (int64_t)blk * kCpBlk;
     const int nt = (int)min((int64_t)kCpBlk, L - t0);
-    // C rows of the block (zeros past the end of the segment), 16 bytes at a time
+    // C rows of the block (zeros past the end of the segment), 16 bytes per asynchronous copy,
+    // all in flight at once
     const int cv = N / 8;
     for (int i = tid; i < kCpBlk * cv; i += blockDim.x) {
         const int r = i / cv, c = i % cv;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (r < nt) v = reinterpret_cast<const uint4 *>(Cm + ((((int64_t)b * L + t0 + r) * G + g) * N))[c];
-        *reinterpret_cast<uint4 *>(ct + r * ld + 8 * c) = v;
+        __nv_bfloat16 *dst = ct + r * ld + 8 * c;
+        if (r < nt) {
+            const __nv_bfloat16 *srcp = Cm + ((((int64_t)b * L + t0 + r) * G + g) * N) + 8 * c;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                         "l"(srcp)
+                         : "memory");
+        } else {
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+        }
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
     block_decay_factors(dt, A[h], bsum + ((int64_t)b * H + h) * nblk, blk, L, H, b, h, cum);
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
 
     const uint32_t ct_base = (uint32_t)__cvta_generic_to_shared(ct), st_base = (uint32_t)__cvta_generic_to_shared(st);
     // ldmatrix row addresses: A (16 x 16 of C, rows 16 warp ..), B (two 8 x 16 tiles of S_in)
@@ -143,14 +153,28 @@ __global__ void __launch_bounds__(256)
     const float *srow = s_in + ((int64_t)b * H + h) * P * N;
     for (int pc = 0; pc < P; pc += 64) {
         __syncthreads();  // the previous chunk's S_in tile has been read
-        for (int i = tid; i < 64 * (N / 4); i += blockDim.x) {
-            const int r = i / (N / 4), c = i % (N / 4);
-            const float4 v = reinterpret_cast<const float4 *>(srow + (int64_t)(pc + r) * N)[c];
-            __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
-            uint2 pk;
-            pk.x = *reinterpret_cast<uint32_t *>(&lo);
-            pk.y = *reinterpret_cast<uint32_t *>(&hi);
-            *reinterpret_cast<uint2 *>(st + r * ld + 4 * c) = pk;
+        // 64 rows x N fp32 of S_in to bf16: each thread's (at most 16) loads are issued
+        // before any of them is converted
+        {
+            const int per = 64 * (N / 4);  // float4 vectors in the chunk, a multiple of 256 / 16
+            float4 v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int i = tid + u * 256;
+                if (i < per) v[u] = reinterpret_cast<const float4 *>(srow + (int64_t)pc * N)[i];
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int i = tid + u * 256;
+                if (i < per) {
+                    const int r = i / (N / 4), c = i % (N / 4);
+                    __nv_bfloat162 lo = __floats2bfloat162_rn(v[u].x, v[u].y), hi = __floats2bfloat162_rn(v[u].z, v[u].w);
+                    uint2 pk;
+                    pk.x = *reinterpret_cast<uint32_t *>(&lo);
+                    pk.y = *reinterpret_cast<uint32_t *>(&hi);
+                    *reinterpret_cast<uint2 *>(st + r * ld + 4 * c) = pk;
+                }
+            }
         }
         __syncthreads();
         float acc[8][4];

@@ -23,6 +23,30 @@ namespace {
 constexpr int kVThreads = 256;
 constexpr int kMaxVec = 2;  // float4 vectors per lane per state row: N <= 256
 
+// Sums of 8 values across the 32 lanes of a warp at once: the halves are exchanged and
+// added (xor 16, 8, 4: 4 + 2 + 1 shuffles) so that lane l ends with value (l >> 2) & 7
+// summed over 8 lanes, then the 4 lanes of each group finish with xor 2 and xor 1. Each
+// value is summed over the same pairs, in the same order, as the full butterfly
+// (xor 16, 8, 4, 2, 1) on that value alone.
+__device__ __forceinline__ float reduce8(const float (&v)[8], int lane) {
+    const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
+    float a[4], c[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float send = h16 ? v[i] : v[i + 4], keep = h16 ? v[i + 4] : v[i];
+        a[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float send = h8 ? a[i] : a[i + 2], keep = h8 ? a[i + 2] : a[i];
+        c[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    float r = (h4 ? c[1] : c[0]) + __shfl_xor_sync(0xffffffffu, h4 ? c[0] : c[1], 4);
+    r += __shfl_xor_sync(0xffffffffu, r, 2);
+    r += __shfl_xor_sync(0xffffffffu, r, 1);
+    return r;
+}
+
 // grid (H, B). Warp w advances rows p = w, w + 8, ...; lane owns float4 vectors
 // v = lane + 32 j of the row. Shared memory: B, C (K x N), x (K x P), dt, decay (K).
 template <typename T>
@@ -67,34 +91,42 @@ __global__ void __launch_bounds__(kVThreads)
             const int v = lane + 32 * j;
             s[j] = v < nv ? src[v] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        for (int k = 0; k < K; ++k) {
-            const float dk = dec[k];
-            const float xk = xsm[k * P + p];
-            const float dx = dts[k] * xk;
-            const float4 *bk = reinterpret_cast<const float4 *>(bsm + k * N);
-            const float4 *ck = reinterpret_cast<const float4 *>(csm + k * N);
-            float4 *dst = states_out ? reinterpret_cast<float4 *>(states_out + ((((int64_t)b * K + k) * H + h) * P + p) * N)
-                                     : nullptr;
-            float part = 0.f;
+        // Tokens in groups of 8: each token's dot product with C is kept as per-lane partials
+        // and the 8 of a group are reduced together (reduce8), so the sequential chain per
+        // token is the state update alone.
+        for (int k0 = 0; k0 < K; k0 += 8) {
+            float part[8];
 #pragma unroll
-            for (int j = 0; j < kMaxVec; ++j) {
-                const int v = lane + 32 * j;
-                if (v < nv) {
-                    const float4 bb = bk[v], cc = ck[v];
-                    s[j].x = fmaf(dk, s[j].x, dx * bb.x);
-                    s[j].y = fmaf(dk, s[j].y, dx * bb.y);
-                    s[j].z = fmaf(dk, s[j].z, dx * bb.z);
-                    s[j].w = fmaf(dk, s[j].w, dx * bb.w);
-                    part = fmaf(s[j].x, cc.x, part);
-                    part = fmaf(s[j].y, cc.y, part);
-                    part = fmaf(s[j].z, cc.z, part);
-                    part = fmaf(s[j].w, cc.w, part);
-                    if (states_out) __stcs(dst + v, s[j]);
+            for (int kk = 0; kk < 8; ++kk) {
+                const int k = k0 + kk;
+                part[kk] = 0.f;
+                if (k >= K) continue;  // warp-uniform
+                const float dk = dec[k];
+                const float dx = dts[k] * xsm[k * P + p];
+                const float4 *bk = reinterpret_cast<const float4 *>(bsm + k * N);
+                const float4 *ck = reinterpret_cast<const float4 *>(csm + k * N);
+                float4 *dst = states_out ? reinterpret_cast<float4 *>(states_out + ((((int64_t)b * K + k) * H + h) * P + p) * N)
+                                         : nullptr;
+#pragma unroll
+                for (int j = 0; j < kMaxVec; ++j) {
+                    const int v = lane + 32 * j;
+                    if (v < nv) {
+                        const float4 bb = bk[v], cc = ck[v];
+                        s[j].x = fmaf(dk, s[j].x, dx * bb.x);
+                        s[j].y = fmaf(dk, s[j].y, dx * bb.y);
+                        s[j].z = fmaf(dk, s[j].z, dx * bb.z);
+                        s[j].w = fmaf(dk, s[j].w, dx * bb.w);
+                        part[kk] = fmaf(s[j].x, cc.x, part[kk]);
+                        part[kk] = fmaf(s[j].y, cc.y, part[kk]);
+                        part[kk] = fmaf(s[j].z, cc.z, part[kk]);
+                        part[kk] = fmaf(s[j].w, cc.w, part[kk]);
+                        if (states_out) __stcs(dst + v, s[j]);
+                    }
                 }
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-            if (lane == 0) store_as(y + (((int64_t)b * K + k) * H + h) * P + p, part + Dh * xk);
+            const float tot = reduce8(part, lane);
+            const int k = k0 + (lane >> 2);
+            if ((lane & 3) == 0 && k < K) store_as(y + (((int64_t)b * K + k) * H + h) * P + p, tot + Dh * xsm[k * P + p]);
         }
     }
 }
@@ -104,9 +136,9 @@ __global__ void __launch_bounds__(kVThreads)
 // A row whose count is outside 0..K is filled with quiet NaN.
 template <typename T>
 __global__ void __launch_bounds__(kVThreads)
-    k_advance(const float *__restrict__ h0, const T *__restrict__ x, const T *__restrict__ dt,
-              const float *__restrict__ A, const T *__restrict__ Bm, const int32_t *__restrict__ accepted,
-              int K, int H, int P, int G, int N, float *__restrict__ h_keep) {
+    k_advance(const float *h0, const T *__restrict__ x, const T *__restrict__ dt, const float *__restrict__ A,
+              const T *__restrict__ Bm, const int32_t *__restrict__ accepted, int K, int H, int P, int G, int N,
+              float *h_keep) {  // h_keep may be h0 (in place): each row is read before it is written, by one warp
     extern __shared__ float sm[];
     const int h = blockIdx.x, b = blockIdx.y, g = h / (H / G);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
