@@ -191,9 +191,8 @@ __device__ __forceinline__ unsigned long long now_ns() {
 // Bounded wait on a barrier phase. Returns false (and raises the abort flag and the
 // status word) when the phase does not complete within kWaitNs or another thread of
 // the CTA has already aborted.
-__device__ __noinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                        int *status) {
-    if (mbar_try(bar, parity)) return true;
+__device__ __noinline__ bool wait_phase_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                             int *status) {
     const unsigned long long t0 = now_ns();
     for (;;) {
         if (mbar_try_sleep(bar, parity)) return true;
@@ -204,6 +203,13 @@ __device__ __noinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile
             return false;
         }
     }
+}
+
+// The common case (the phase has completed) stays inline: an out-of-line call costs a stack
+// frame in local memory, which shares the L1 / shared-memory port with everything else.
+__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *status) {
+    if (mbar_try(bar, parity)) return true;
+    return wait_phase_slow(bar, parity, abort_flag, status);
 }
 
 __device__ __forceinline__ void fence_proxy_async() {
