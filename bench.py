@@ -427,7 +427,7 @@ def aux_main(args):
     yseg = torch.zeros(Bsz, Ls, H, P, dtype=torch.bfloat16, device=dev)
     ms = timed(lambda: ssd.ssd_cp_correct(g["dt"], g["A"], g["C"], bd, s_in, yseg, stream=stream))
     flops = 2.0 * Bsz * Ls * H * P * N
-    emit("k_correct_mma", f"long_n256 segment 1/{R}", ms,
+    emit("k_correct_tc", f"long_n256 segment 1/{R}", ms,
          2 * Bsz * Ls * H * P * 2 + Bsz * Ls * G * N * 2 + Bsz * Ls * H * 2 + Bsz * H * P * N * 4, 1,
          flops=flops, tflops=flops / (ms * 1e-3) / 1e12)
     return 0

@@ -261,12 +261,16 @@ ssd_status_t ssd_cp_combine(const ssd_shape_t *shape, int64_t nranks, int64_t ra
  *   block_decay   [B, H, ceil(L/128)] from ssd_cp_decay on the same segment
  *   s_in          [B, H, P, N] fp32 from ssd_cp_combine
  *   y             [B, L, H, P] dtype, read and written (y += the incoming state's term)
- * bf16 inputs with headdim % 64 == 0 and dstate % 16 == 0 run on tensor cores (S_in
- * rounded to bf16, fp32 accumulation); other shapes and fp32 inputs in fp32 on CUDA cores.
+ *   status        int32 device word or NULL: bit 0 is set (never cleared) if a bounded
+ *                 device-side wait ran out, in which case y is incomplete; zero it beforehand
+ * bf16 inputs run on tensor cores with S_in rounded to bf16 and fp32 accumulation: tcgen05
+ * when headdim == 64, dstate % 64 == 0 and each group has an even number of heads, mma.sync
+ * when headdim % 64 == 0 and dstate % 16 == 0. Other shapes and fp32 inputs run in fp32 on
+ * CUDA cores.
  */
 ssd_status_t ssd_cp_correct(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *dt, const float *A,
                             const void *Cm, const float *block_decay, const float *s_in, void *y,
-                            void *stream);
+                            int32_t *status, void *stream);
 
 #ifdef __cplusplus
 }

@@ -49,7 +49,7 @@ _SIGS = {
     "ssd_decode_step": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 9, ctypes.c_int),
     "ssd_cp_decay": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 5, ctypes.c_int),
     "ssd_cp_combine": ([ctypes.POINTER(ShapeT), _i64, _i64] + [_vp] * 5, ctypes.c_int),
-    "ssd_cp_correct": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 7, ctypes.c_int),
+    "ssd_cp_correct": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 8, ctypes.c_int),
 }
 
 CP_BLOCK = 128  # SSD_CP_BLOCK: tokens per decay block
@@ -242,13 +242,15 @@ def ssd_cp_combine(states, totals, rank, *, s_in=None, h_final=None, want_final=
     return s_in, h_final
 
 
-def ssd_cp_correct(dt, A, C, block_decay, s_in, y, *, stream=None):
-    """y += exp(cumulative dt*A from the segment start) * C S_in^T, in place; returns y."""
-    dev = _dev(dt, A, C, block_decay, s_in, y)
+def ssd_cp_correct(dt, A, C, block_decay, s_in, y, *, status=None, stream=None):
+    """y += exp(cumulative dt*A from the segment start) * C S_in^T, in place; returns y.
+    status: optional int32 device tensor (one element, zeroed by the caller); bit 0 is set if a
+    bounded device-side wait ran out."""
+    dev = _dev(dt, A, C, block_decay, s_in, y, status)
     Bsz, L, H, P = y.shape
     G, N = C.shape[2], C.shape[3]
     shape = ShapeT(Bsz, L, H, P, G, N)
     st = lib().ssd_cp_correct(ctypes.byref(shape), _dtype_code(y), _ptr(dt), _ptr(A), _ptr(C), _ptr(block_decay),
-                              _ptr(s_in), _ptr(y), _stream(dev, stream))
+                              _ptr(s_in), _ptr(y), _ptr(status), _stream(dev, stream))
     _check(st, "ssd_cp_correct")
     return y

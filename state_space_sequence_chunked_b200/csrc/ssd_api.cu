@@ -259,7 +259,7 @@ SSD_API ssd_status_t ssd_cp_combine(const ssd_shape_t *shape, int64_t nranks, in
 
 SSD_API ssd_status_t ssd_cp_correct(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *dt, const float *A,
                                     const void *Cm, const float *block_decay, const float *s_in, void *y,
-                                    void *stream) {
+                                    int32_t *status, void *stream) {
     ssd_status_t st = check_shape(shape);
     if (st != SSD_OK) return st;
     if ((st = check_dtype(dtype)) != SSD_OK) return st;
@@ -268,6 +268,7 @@ SSD_API ssd_status_t ssd_cp_correct(const ssd_shape_t *shape, ssd_dtype_t dtype,
     const void *ptrs[] = {dt, A, Cm, block_decay, s_in, y};
     for (const void *q : ptrs)
         if (!aligned16(q)) return SSD_ERR_ALIGNMENT;
-    return from_cuda(cp_correct_launch(make_cp(shape, dtype), dt, A, Cm, block_decay, s_in, y,
+    if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return SSD_ERR_ALIGNMENT;
+    return from_cuda(cp_correct_launch(make_cp(shape, dtype), dt, A, Cm, block_decay, s_in, y, status,
                                        static_cast<cudaStream_t>(stream)));
 }

@@ -16,6 +16,8 @@
 //   k_block_decay   per 128-token block sums of dt A (coalesced over heads)
 //   k_total_decay   Lambda = the block sums added in order
 //   k_combine       the exclusive scan over ranks (elementwise over the state)
+//   k_correct_tc    (ssd_cp_tc.cu) the correction on tcgen05 for bf16, P = 64, N % 64 == 0,
+//                   an even number of heads per group
 //   k_correct_mma   the correction with bf16 mma.sync tiles (128 tokens x 64 columns of P)
 //   k_correct_simt  the same in fp32 on CUDA cores (fp32 inputs, or shapes the tiles do not fit)
 #include "ssd_internal.cuh"
@@ -294,9 +296,10 @@ cudaError_t cp_combine_launch(const CpProblem &p, int R, int rank, const float *
 bool cp_correct_uses_mma(const CpProblem &p) { return p.dtype == SSD_BF16 && p.P % 64 == 0 && p.N % 16 == 0; }
 
 cudaError_t cp_correct_launch(const CpProblem &p, const void *dt, const float *A, const void *Cm, const float *bsum,
-                              const float *s_in, void *y, cudaStream_t s) {
+                              const float *s_in, void *y, int *status, cudaStream_t s) {
     const int nblk = cp_nblk(p.L);
     if (nblk == 0) return cudaSuccess;
+    if (cp_correct_uses_tc(p)) return cp_correct_tc_launch(p, dt, A, Cm, bsum, s_in, y, status, s);
     dim3 grid((unsigned)nblk, (unsigned)p.H, (unsigned)p.B);
     const int H = (int)p.H, P = (int)p.P, G = (int)p.G, N = (int)p.N;
     cudaError_t e;

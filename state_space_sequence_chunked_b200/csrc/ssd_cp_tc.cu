@@ -1,0 +1,237 @@
+// The context-parallel state-to-output correction on tcgen05 tensor cores.
+//
+// For a segment of the sequence and the state S_in entering it (the exclusive scan of the
+// ranks' end states, "序列并行" in the Mamba-2 SSD write-up), every token's output gains
+//     y_t[h, :] += exp(sum_{s <= t in segment} dt_s A_h) * S_in[h] C_t
+// which is step 4 of the chunked algorithm ("SSD 算法：分块和状态传递") for the incoming state.
+// Over one 128-token block and two heads of one group it is a single matrix product
+//     Y[t, (h, p)] = sum_n C[t, n] S_in[h, p, n]        (M = 128 tokens, N = 2 x 64, K = dstate)
+// followed by a per-(token, head) scaling. One CTA per (block, head pair, batch row):
+//   - TMA brings the block's C (K-major, 128-byte swizzle, 64-column panels) and the two
+//     heads' y tiles;
+//   - the 256 threads write S_in, converted to bf16, in the same K-major swizzled layout;
+//   - one thread issues dstate / 16 MMAs (M = 128, N = 128) into a TMEM accumulator;
+//   - warps 0-1 form the decay factors of the two heads meanwhile;
+//   - each warp reads its TMEM lane quarter for one head, updates the y tile in shared
+//     memory, and one thread stores both tiles with TMA.
+// Every wait is bounded; a wait that runs out sets bit 0 of *status (when given) and the CTA
+// skips the rest of its work.
+#include "tc_ptx.cuh"
+
+namespace ssd {
+namespace cpt {
+using namespace tc;
+
+constexpr int kBlk = 128;      // tokens per CTA
+constexpr int kP = 64;         // head dimension this kernel takes
+constexpr int kPanel = 16384;  // one 64-column panel of a 128-row K-major tile, bytes
+constexpr int kThreads = 256;
+
+struct Params {
+    const __nv_bfloat16 *dt;
+    const float *A, *bsum, *s_in;
+    int *status;
+    long long L;
+    int H, G, N, nblk, pairs_per_group;
+};
+
+// Shared memory (after 1024-byte alignment): C tile [N/64 panels], S_in tile [N/64 panels],
+// y tiles [2][128 rows x 128 B], cum [2][128] fp32, barriers, TMEM base, abort flag.
+__host__ __device__ constexpr int smem_bytes(int N) { return 2 * (N / 64) * kPanel + 2 * kPanel + 2 * kBlk * 4 + 64; }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_correct_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y, const Params prm) {
+    extern __shared__ unsigned char cpt_raw[];
+    unsigned char *sm =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(cpt_raw) + 1023) & ~uintptr_t(1023));
+    const int N = prm.N, npan = N / 64;
+    unsigned char *c_tile = sm;
+    unsigned char *s_tile = sm + npan * kPanel;
+    unsigned char *y_tile = sm + 2 * npan * kPanel;  // [2][16 KB]
+    float *cum = reinterpret_cast<float *>(y_tile + 2 * kPanel);
+    uint64_t *ld_bar = reinterpret_cast<uint64_t *>(cum + 2 * kBlk);
+    uint64_t *mma_bar = ld_bar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_bar + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int local_status = 0;
+    int *status = prm.status ? prm.status : &local_status;
+
+    const int blk = blockIdx.x, b = blockIdx.z;
+    const int g = blockIdx.y / prm.pairs_per_group, pr = blockIdx.y % prm.pairs_per_group;
+    const int hpg = prm.H / prm.G, h0 = g * hpg + 2 * pr;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long L = prm.L, t0 = (long long)blk * kBlk;
+
+    if (tid == 0) {
+        mbar_init(ld_bar, 1);
+        mbar_init(mma_bar, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(128)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (tid == 0) {  // C panels of the block and the two heads' y tiles
+        mbar_arrive_tx(ld_bar, (uint32_t)(npan * kPanel + 2 * kPanel));
+        for (int pn = 0; pn < npan; ++pn) tma_load_4d(c_tile + pn * kPanel, &tm_c, ld_bar, 64 * pn, g, (int)t0, b);
+        for (int e = 0; e < 2; ++e) tma_load_4d(y_tile + e * kPanel, &tm_y, ld_bar, 0, h0 + e, (int)t0, b);
+    }
+    // S_in of the two heads -> bf16, K-major: row r = 64 e + p, 16-byte chunk (n / 8) in panel n / 64
+    {
+        const float *src = prm.s_in + ((long long)b * prm.H + h0) * kP * N;  // the two heads are adjacent
+        // chunks = 128 * N / 8 is a multiple of 4 * kThreads: four chunks' loads are issued per
+        // thread before any of them is converted
+        const int chunks = kBlk * (N / 8);
+        for (int i0 = tid; i0 < chunks; i0 += 4 * kThreads) {
+            float4 lo[4], hi[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * kThreads, r = i / (N / 8), cc = i % (N / 8);
+                lo[u] = reinterpret_cast<const float4 *>(src + (long long)r * N)[2 * cc];
+                hi[u] = reinterpret_cast<const float4 *>(src + (long long)r * N)[2 * cc + 1];
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * kThreads, r = i / (N / 8), cc = i % (N / 8);
+                uint4 o;
+                o.x = pack_bf16(lo[u].x, lo[u].y);
+                o.y = pack_bf16(lo[u].z, lo[u].w);
+                o.z = pack_bf16(hi[u].x, hi[u].y);
+                o.w = pack_bf16(hi[u].z, hi[u].w);
+                *reinterpret_cast<uint4 *>(s_tile + (cc >> 3) * kPanel + swz(r, cc & 7)) = o;
+            }
+        }
+    }
+    fence_proxy_async();  // the generic-proxy writes of S_in are visible to the tensor cores
+    __syncthreads();
+    if (tid == 0) {
+        if (wait_phase(ld_bar, 0, abort_flag, status)) {
+            tc_fence_after();
+            const uint32_t ca = smem_u32(c_tile), sa = smem_u32(s_tile);
+            constexpr uint32_t kId = idesc(128, 128, false, false);
+#pragma unroll 1
+            for (int kk = 0; kk < N / 16; ++kk) {
+                const uint32_t off = (uint32_t)((kk >> 2) * kPanel + (kk & 3) * 32);
+                mma_ss(tmem, sdesc(ca + off, 16, 1024), sdesc(sa + off, 16, 1024), kId, kk > 0);
+            }
+            mma_commit(mma_bar);
+        }
+    }
+    if (warp < 2) {  // decay factors exp(cumulative dt A) of head h0 + warp for the block's tokens
+        const int h = h0 + warp;
+        const float a = prm.A[h];
+        const float *bs = prm.bsum + ((long long)b * prm.H + h) * prm.nblk;
+        float pre = 0.f;
+        for (int k = lane; k < blk; k += 32) pre += bs[k];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) pre += __shfl_xor_sync(0xffffffffu, pre, o);
+        const long long tt = t0 + 4 * lane;
+        float v[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) v[m] = tt + m < L ? __bfloat162float(prm.dt[((long long)b * L + tt + m) * prm.H + h]) * a : 0.f;
+        v[1] += v[0];
+        v[2] += v[1];
+        v[3] += v[2];
+        float incl = v[3];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
+        }
+        const float excl = incl - v[3] + pre;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) cum[warp * kBlk + 4 * lane + m] = expf(excl + v[m]);
+    }
+    __syncthreads();
+    // epilogue: warp w reads TMEM lane quarter w % 4 (tokens 32 (w % 4) ..) for head w / 4
+    const bool ok = wait_warp(mma_bar, 0, abort_flag, status) && wait_warp(ld_bar, 0, abort_flag, status);
+    if (ok) {
+        tc_fence_after();
+        const int q = warp & 3, e = warp >> 2, row = 32 * q + lane;
+        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + 64 * e;
+        const float w = cum[e * kBlk + row];
+        unsigned char *yr = y_tile + e * kPanel;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+            uint32_t acc[32];
+            tmem_ld32(taddr + 32 * half, acc);
+            tmem_wait_ld(acc);
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {  // 16-byte chunks 4 half + c4 of the row (8 columns each)
+                uint4 *pv = reinterpret_cast<uint4 *>(yr + swz(row, 4 * half + c4));
+                const uint4 old = *pv;
+                const uint32_t ov[4] = {old.x, old.y, old.z, old.w};
+                uint32_t nv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float a0 = __uint_as_float(acc[8 * c4 + 2 * u]), a1 = __uint_as_float(acc[8 * c4 + 2 * u + 1]);
+                    nv[u] = pack_bf16(fmaf(w, a0, bf16_lo(ov[u])), fmaf(w, a1, bf16_hi(ov[u])));
+                }
+                *pv = make_uint4(nv[0], nv[1], nv[2], nv[3]);
+            }
+        }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && ok && !*abort_flag) {
+        for (int e = 0; e < 2; ++e) tma_store_4d(&tm_y, y_tile + e * kPanel, 0, h0 + e, (int)t0, b, policy_evict_first());
+        bulk_commit();
+        bulk_wait_all();
+    }
+    if (warp == 0) {
+        if (lane == 0 && !ok) {  // MMAs still in flight must finish before TMEM is released
+            const unsigned long long w0 = now_ns();
+            while (!mbar_try(mma_bar, 0) && now_ns() - w0 < kWaitNs) {
+            }
+        }
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128) : "memory");
+    }
+}
+
+}  // namespace cpt
+
+bool cp_correct_uses_tc(const CpProblem &p) {
+    return p.dtype == SSD_BF16 && p.P == cpt::kP && p.N % 64 == 0 && p.N <= 256 && (p.H / p.G) % 2 == 0 &&
+           p.L < (1ll << 31);
+}
+
+cudaError_t cp_correct_tc_launch(const CpProblem &p, const void *dt, const float *A, const void *Cm, const float *bsum,
+                                 const float *s_in, void *y, int *status, cudaStream_t s) {
+    using namespace cpt;
+    const int nblk = cp_nblk(p.L);
+    if (nblk == 0) return cudaSuccess;
+    CUtensorMap tmc, tmy;
+    if (!tc::encode_4d(&tmc, Cm, p.N, p.G, p.L, p.B) || !tc::encode_4d(&tmy, y, kP, p.H, p.L, p.B))
+        return cudaErrorInvalidValue;
+    Params prm;
+    prm.dt = static_cast<const __nv_bfloat16 *>(dt);
+    prm.A = A;
+    prm.bsum = bsum;
+    prm.s_in = s_in;
+    prm.status = status;
+    prm.L = p.L;
+    prm.H = (int)p.H;
+    prm.G = (int)p.G;
+    prm.N = (int)p.N;
+    prm.nblk = nblk;
+    prm.pairs_per_group = (int)(p.H / p.G / 2);
+    const int smem = smem_bytes((int)p.N) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_correct_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)nblk, (unsigned)(p.G * prm.pairs_per_group), (unsigned)p.B);
+    k_correct_tc<<<grid, kThreads, smem, s>>>(tmc, tmy, prm);
+    return cudaGetLastError();
+}
+
+}  // namespace ssd

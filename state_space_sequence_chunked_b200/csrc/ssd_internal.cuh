@@ -64,8 +64,11 @@ cudaError_t cp_block_decay_launch(const CpProblem &p, const void *dt, const floa
 cudaError_t cp_combine_launch(const CpProblem &p, int R, int rank, const float *states, const float *totals,
                               float *s_in, float *h_final, cudaStream_t s);
 bool cp_correct_uses_mma(const CpProblem &p);
+bool cp_correct_uses_tc(const CpProblem &p);
+cudaError_t cp_correct_tc_launch(const CpProblem &p, const void *dt, const float *A, const void *Cm, const float *bsum,
+                                 const float *s_in, void *y, int *status, cudaStream_t s);
 cudaError_t cp_correct_launch(const CpProblem &p, const void *dt, const float *A, const void *Cm, const float *bsum,
-                              const float *s_in, void *y, cudaStream_t s);
+                              const float *s_in, void *y, int *status, cudaStream_t s);
 
 // ---- element access ---------------------------------------------------------------
 __device__ __forceinline__ float to_f32(float v) { return v; }

@@ -41,11 +41,9 @@
 // the next block's B and C load as soon as the products that read them are done. Every
 // wait is bounded: on timeout the CTA raises a status word in the workspace, drains its
 // own TMA loads and MMAs, frees TMEM and returns.
-#include <cuda.h>
-
 #include <algorithm>
 
-#include "ssd_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace ssd {
 namespace tc {
@@ -55,7 +53,6 @@ constexpr int kP = 64;   // head dimension handled by this path
 constexpr int kThreads = 384;
 constexpr int kWarpTma = 0, kWarpG = 1, kWarpDs = 2, kWarpYs = 3, kWarpE = 8;  // warps 4-7: T
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
 
 template <int N>
 struct Cfg {
@@ -130,265 +127,6 @@ __device__ __forceinline__ Share share_of(long long total, int nc, int i, int G)
     return s;
 }
 
-// ---------------------------------------------------------------------------------
-// PTX wrappers
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// As mbar_try, but a thread whose phase is not complete sleeps (up to the hint, in ns)
-// until it completes instead of returning at once, so waiting warps take no issue slots
-// from the warps that do the work.
-__device__ __forceinline__ bool mbar_try_sleep(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(0x989680u)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ unsigned long long now_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Bounded wait on a barrier phase. Returns false (and raises the abort flag and the
-// status word) when the phase does not complete within kWaitNs or another thread of
-// the CTA has already aborted.
-__device__ __noinline__ bool wait_phase_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                             int *status) {
-    const unsigned long long t0 = now_ns();
-    for (;;) {
-        if (mbar_try_sleep(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (now_ns() - t0 > kWaitNs) {
-            *abort_flag = 1;
-            atomicOr(status, 1);
-            return false;
-        }
-    }
-}
-
-// The common case (the phase has completed) stays inline: an out-of-line call costs a stack
-// frame in local memory, which shares the L1 / shared-memory port with everything else.
-__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *status) {
-    if (mbar_try(bar, parity)) return true;
-    return wait_phase_slow(bar, parity, abort_flag, status);
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1,
-                                            int c2, int c3) {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
-        "[%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-        : "memory");
-}
-
-// L2 policies: B and C tiles are read by every head of their group, so they should stay;
-// x is read once and y written once, so they should go first.
-__device__ __forceinline__ uint64_t policy_evict_last() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-__device__ __forceinline__ uint64_t policy_evict_first() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-__device__ __forceinline__ void tma_load_4d_hint(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1,
-                                                 int c2, int c3, uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, "
-        "%4, %5, %6}], [%2], %7;" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
-        : "memory");
-}
-__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void *src, int c0, int c1, int c2,
-                                             int c3, uint64_t policy) {
-    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3, %4, %5}], [%1], %6;" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-// Shared-memory matrix descriptor, 128-byte swizzle (sm100 format: version 1).
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    uint64_t d = 0;
-    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-    d |= (uint64_t)1 << 46;
-    d |= (uint64_t)2 << 61;
-    return d;
-}
-
-// Instruction descriptor, kind::f16 with bf16 operands and fp32 accumulation.
-__host__ __device__ constexpr uint32_t idesc(int M, int N, bool a_mn, bool b_mn) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
-           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-        "l"(a), "l"(b), "r"(id), "r"(acc)
-        : "memory");
-}
-__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t id, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-        "r"(a_tmem), "l"(b), "r"(id), "r"(acc)
-        : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_u32(bar))
-                 : "memory");
-}
-
-#define SSD_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), \
-                  "=r"(r[i + 6]), "=r"(r[i + 7])
-// 32 consecutive columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : SSD_R8(0), SSD_R8(8), SSD_R8(16), SSD_R8(24)
-        : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : SSD_R8(0)
-                 : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-        "%14, %15}, [%16];"
-        : SSD_R8(0), SSD_R8(8)
-        : "r"(taddr));
-}
-#undef SSD_R8
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-// The same wait, with the registers of an earlier tcgen05.ld as operands, so that the
-// compiler cannot move a use of them above it (needed when other loads are in flight).
-#define SSD_W8(i) "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]), \
-                  "+r"(r[i + 6]), "+r"(r[i + 7])
-__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;" : SSD_W8(0), SSD_W8(8), SSD_W8(16), SSD_W8(24)::"memory");
-}
-#undef SSD_W8
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-        "%14, %15, %16};" ::"r"(taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    uint32_t r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-// Packed fp32 pairs (sm_100): s = g s + d r on two lanes of the state at once, and
-// w (a, b) rounded to a bf16 pair.
-__device__ __forceinline__ void fma2_state(float &s0, float &s1, float g, float d, uint32_t r0, uint32_t r1) {
-    asm("{\n\t.reg .b64 s, q, gg, dd;\n\t"
-        "mov.b64 s, {%0, %1};\n\tmov.b64 q, {%4, %5};\n\t"
-        "mov.b64 gg, {%2, %2};\n\tmov.b64 dd, {%3, %3};\n\t"
-        "mul.rn.f32x2 q, q, dd;\n\tfma.rn.f32x2 s, gg, s, q;\n\t"
-        "mov.b64 {%0, %1}, s;\n\t}"
-        : "+f"(s0), "+f"(s1)
-        : "f"(g), "f"(d), "r"(r0), "r"(r1));
-}
-__device__ __forceinline__ uint32_t scale2_bf16(float w, float a, float b) {
-    uint32_t o;
-    asm("{\n\t.reg .b64 v, ww;\n\t.reg .f32 lo, hi;\n\t"
-        "mov.b64 v, {%2, %3};\n\tmov.b64 ww, {%1, %1};\n\t"
-        "mul.rn.f32x2 v, v, ww;\n\t"
-        "mov.b64 {lo, hi}, v;\n\tcvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
-        : "=r"(o)
-        : "f"(w), "f"(a), "f"(b));
-    return o;
-}
-__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-
-// Byte offset of 16-byte chunk `c` of row `r` in a 128-byte-swizzled tile (128 B rows).
-__device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
-
-// Warp-uniform bounded wait: every lane polls (each gets the acquire), and the
-// warp agrees on the outcome, so a timeout never leaves part of a warp behind
-// at a warp-collective instruction. Call only from warp-uniform control flow.
-__device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *status) {
-    const bool ok = wait_phase(bar, parity, abort_flag, status);
-    return __all_sync(0xffffffffu, ok);
-}
-
-// Within-block inclusive cumsum of dts[i] * a2, i = 0..127, by one warp on its own
-// (lane handles i = lane + 32 m). v[m] is the value at index 32 m + lane; the
-// block total is returned. Every warp runs the same sequence of operations, so
-// every warp gets bit-identical values.
 // ---------------------------------------------------------------------------------
 
 // Exact form of G' for one warp's 32 rows (lane quarter qtr): every element of the causal
@@ -997,43 +735,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------------------------
 // host side
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;  // process-wide cache of the driver entry point
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// [B, L, X, inner] bf16 tensor, box {64, 1, rows, 1}, 128-byte swizzle.
-bool encode_4d(CUtensorMap *m, const void *base, int64_t inner, int64_t X, int64_t L, int64_t B, int rows = kQ) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)X, (cuuint64_t)L, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)(inner * 2), (cuuint64_t)(X * inner * 2),
-                                   (cuuint64_t)(L * X * inner * 2)};
-    const cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int num_sms() {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    return n;
-}
 
 template <int N>
 cudaError_t launch(const FwdProblem &p, int *status, int *flags, float *handover, int grid, cudaStream_t s) {
