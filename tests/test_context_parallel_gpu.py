@@ -30,13 +30,16 @@ def emulate(g, R, chunk):
         segs.append((lo, hi)); ys.append(y); hs.append(h); bds.append(bd); tots.append(tot)
     states, totals = torch.stack(hs), torch.stack(tots)
     ends = []
+    status = torch.zeros(4, dtype=torch.int32, device=g["x"].device)
     for r in range(R):
         lo, hi = segs[r]
         s_in, h_end = ssd.ssd_cp_combine(states, totals, r)
         if r > 0:
-            ssd.ssd_cp_correct(g["dt"][:, lo:hi].clone(), g["A"], g["C"][:, lo:hi].clone(), bds[r], s_in, ys[r])
+            ssd.ssd_cp_correct(g["dt"][:, lo:hi].clone(), g["A"], g["C"][:, lo:hi].clone(), bds[r], s_in, ys[r],
+                               status=status)
         ends.append(h_end)
     torch.cuda.synchronize()
+    assert int(status[0].item()) == 0, "a bounded wait of the correction ran out"
     return torch.cat(ys, dim=1), ends
 
 
