@@ -6,16 +6,19 @@
 // which is step 4 of the chunked algorithm ("SSD 算法：分块和状态传递") for the incoming state.
 // Over one 128-token block and two heads of one group it is a single matrix product
 //     Y[t, (h, p)] = sum_n C[t, n] S_in[h, p, n]        (M = 128 tokens, N = 2 x 64, K = dstate)
-// followed by a per-(token, head) scaling. One CTA per (block, head pair, batch row):
-//   - TMA brings the block's C (K-major, 128-byte swizzle, 64-column panels) and the two
-//     heads' y tiles;
-//   - the 256 threads write S_in, converted to bf16, in the same K-major swizzled layout;
+// followed by a per-(token, head) scaling. A CTA takes one head pair of one batch row and a run
+// of consecutive 128-token blocks, all of which share S_in:
+//   - the 256 threads write S_in once, converted to bf16, K-major with 128-byte swizzle;
+//   - per block, TMA brings C (same layout, 64-column panels) and the two heads' y tiles (two y
+//     buffers: the next block's tiles load while this block's are updated);
 //   - one thread issues dstate / 16 MMAs (M = 128, N = 128) into a TMEM accumulator;
-//   - warps 0-1 form the decay factors of the two heads meanwhile;
-//   - each warp reads its TMEM lane quarter for one head, updates the y tile in shared
+//   - warps 0-1 form the decay factors of the two heads;
+//   - each warp reads its TMEM lane quarter for one head and updates the y tile in shared
 //     memory, and one thread stores both tiles with TMA.
 // Every wait is bounded; a wait that runs out sets bit 0 of *status (when given) and the CTA
 // skips the rest of its work.
+#include <algorithm>
+
 #include "tc_ptx.cuh"
 
 namespace ssd {
@@ -32,12 +35,12 @@ struct Params {
     const float *A, *bsum, *s_in;
     int *status;
     long long L;
-    int H, G, N, nblk, pairs_per_group;
+    int H, G, N, nblk, pairs_per_group, blocks_per_cta;
 };
 
-// Shared memory (after 1024-byte alignment): C tile [N/64 panels], S_in tile [N/64 panels],
-// y tiles [2][128 rows x 128 B], cum [2][128] fp32, barriers, TMEM base, abort flag.
-__host__ __device__ constexpr int smem_bytes(int N) { return 2 * (N / 64) * kPanel + 2 * kPanel + 2 * kBlk * 4 + 64; }
+// Shared memory (after 1024-byte alignment): S_in tile [N/64 panels], C tile [N/64 panels],
+// y tiles [2 buffers][2 heads][128 rows x 128 B], cum [2][128] fp32, barriers, TMEM base, abort.
+__host__ __device__ constexpr int smem_bytes(int N) { return 2 * (N / 64) * kPanel + 4 * kPanel + 2 * kBlk * 4 + 64; }
 
 __global__ void __launch_bounds__(kThreads, 1)
     k_correct_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y, const Params prm) {
@@ -45,25 +48,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char *sm =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(cpt_raw) + 1023) & ~uintptr_t(1023));
     const int N = prm.N, npan = N / 64;
-    unsigned char *c_tile = sm;
-    unsigned char *s_tile = sm + npan * kPanel;
-    unsigned char *y_tile = sm + 2 * npan * kPanel;  // [2][16 KB]
-    float *cum = reinterpret_cast<float *>(y_tile + 2 * kPanel);
-    uint64_t *ld_bar = reinterpret_cast<uint64_t *>(cum + 2 * kBlk);
-    uint64_t *mma_bar = ld_bar + 1;
+    unsigned char *s_tile = sm;
+    unsigned char *c_tile = sm + npan * kPanel;
+    unsigned char *y_tile = sm + 2 * npan * kPanel;  // [2][2][16 KB]
+    float *cum = reinterpret_cast<float *>(y_tile + 4 * kPanel);
+    uint64_t *ld_bar = reinterpret_cast<uint64_t *>(cum + 2 * kBlk);  // [2]: C and y of block i, i % 2
+    uint64_t *mma_bar = ld_bar + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int local_status = 0;
     int *status = prm.status ? prm.status : &local_status;
 
-    const int blk = blockIdx.x, b = blockIdx.z;
+    const int b = blockIdx.z;
     const int g = blockIdx.y / prm.pairs_per_group, pr = blockIdx.y % prm.pairs_per_group;
     const int hpg = prm.H / prm.G, h0 = g * hpg + 2 * pr;
+    const int blk0 = blockIdx.x * prm.blocks_per_cta, nb = min(prm.blocks_per_cta, prm.nblk - blk0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const long long L = prm.L, t0 = (long long)blk * kBlk;
+    const long long L = prm.L;
 
     if (tid == 0) {
-        mbar_init(ld_bar, 1);
+        mbar_init(&ld_bar[0], 1);
+        mbar_init(&ld_bar[1], 1);
         mbar_init(mma_bar, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -78,17 +83,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-
-    if (tid == 0) {  // C panels of the block and the two heads' y tiles
-        mbar_arrive_tx(ld_bar, (uint32_t)(npan * kPanel + 2 * kPanel));
-        for (int pn = 0; pn < npan; ++pn) tma_load_4d(c_tile + pn * kPanel, &tm_c, ld_bar, 64 * pn, g, (int)t0, b);
-        for (int e = 0; e < 2; ++e) tma_load_4d(y_tile + e * kPanel, &tm_y, ld_bar, 0, h0 + e, (int)t0, b);
-    }
-    // S_in of the two heads -> bf16, K-major: row r = 64 e + p, 16-byte chunk (n / 8) in panel n / 64
+    const uint32_t load_bytes = (uint32_t)(npan * kPanel + 2 * kPanel);
+    // C panels and the two heads' y tiles of the CTA's block i, into y buffer i % 2
+    auto issue_loads = [&](int i) {
+        const int t0 = (blk0 + i) * kBlk;
+        uint64_t *bar = &ld_bar[i & 1];
+        mbar_arrive_tx(bar, load_bytes);
+        for (int pn = 0; pn < npan; ++pn) tma_load_4d(c_tile + pn * kPanel, &tm_c, bar, 64 * pn, g, t0, b);
+        for (int e = 0; e < 2; ++e) tma_load_4d(y_tile + ((i & 1) * 2 + e) * kPanel, &tm_y, bar, 0, h0 + e, t0, b);
+    };
+    if (tid == 0 && nb > 0) issue_loads(0);
+    // S_in of the two heads -> bf16, K-major: row r = 64 e + p, 16-byte chunk (n / 8) in panel n / 64.
+    // chunks = 128 N / 8 is a multiple of 4 * kThreads: four chunks' loads are issued per thread
+    // before any of them is converted.
     {
         const float *src = prm.s_in + ((long long)b * prm.H + h0) * kP * N;  // the two heads are adjacent
-        // chunks = 128 * N / 8 is a multiple of 4 * kThreads: four chunks' loads are issued per
-        // thread before any of them is converted
         const int chunks = kBlk * (N / 8);
         for (int i0 = tid; i0 < chunks; i0 += 4 * kThreads) {
             float4 lo[4], hi[4];
@@ -112,85 +121,106 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_proxy_async();  // the generic-proxy writes of S_in are visible to the tensor cores
     __syncthreads();
-    if (tid == 0) {
-        if (wait_phase(ld_bar, 0, abort_flag, status)) {
-            tc_fence_after();
-            const uint32_t ca = smem_u32(c_tile), sa = smem_u32(s_tile);
-            constexpr uint32_t kId = idesc(128, 128, false, false);
-#pragma unroll 1
-            for (int kk = 0; kk < N / 16; ++kk) {
-                const uint32_t off = (uint32_t)((kk >> 2) * kPanel + (kk & 3) * 32);
-                mma_ss(tmem, sdesc(ca + off, 16, 1024), sdesc(sa + off, 16, 1024), kId, kk > 0);
+
+    const int q = warp & 3, e = warp >> 2, row = 32 * q + lane;  // epilogue: TMEM lane quarter, head
+    const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + 64 * e;
+    bool ok = true;
+    int last_mma = -1, last_ld = nb > 0 ? 0 : -1;  // thread 0: the latest block whose MMAs / loads it issued
+    for (int i = 0; i < nb && ok; ++i) {
+        const int blk = blk0 + i;
+        const long long t0 = (long long)blk * kBlk;
+        if (warp < 2) {  // decay factors exp(cumulative dt A) of head h0 + warp over the block's tokens
+            const int h = h0 + warp;
+            const float a = prm.A[h];
+            const float *bs = prm.bsum + ((long long)b * prm.H + h) * prm.nblk;
+            float pre = 0.f;
+            for (int k = lane; k < blk; k += 32) pre += bs[k];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) pre += __shfl_xor_sync(0xffffffffu, pre, o);
+            const long long tt = t0 + 4 * lane;
+            float v[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                v[m] = tt + m < L ? __bfloat162float(prm.dt[((long long)b * L + tt + m) * prm.H + h]) * a : 0.f;
+            v[1] += v[0];
+            v[2] += v[1];
+            v[3] += v[2];
+            float incl = v[3];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float u = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += u;
             }
-            mma_commit(mma_bar);
+            const float excl = incl - v[3] + pre;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) cum[warp * kBlk + 4 * lane + m] = expf(excl + v[m]);
         }
-    }
-    if (warp < 2) {  // decay factors exp(cumulative dt A) of head h0 + warp for the block's tokens
-        const int h = h0 + warp;
-        const float a = prm.A[h];
-        const float *bs = prm.bsum + ((long long)b * prm.H + h) * prm.nblk;
-        float pre = 0.f;
-        for (int k = lane; k < blk; k += 32) pre += bs[k];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) pre += __shfl_xor_sync(0xffffffffu, pre, o);
-        const long long tt = t0 + 4 * lane;
-        float v[4];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) v[m] = tt + m < L ? __bfloat162float(prm.dt[((long long)b * L + tt + m) * prm.H + h]) * a : 0.f;
-        v[1] += v[0];
-        v[2] += v[1];
-        v[3] += v[2];
-        float incl = v[3];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float u = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += u;
-        }
-        const float excl = incl - v[3] + pre;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) cum[warp * kBlk + 4 * lane + m] = expf(excl + v[m]);
-    }
-    __syncthreads();
-    // epilogue: warp w reads TMEM lane quarter w % 4 (tokens 32 (w % 4) ..) for head w / 4
-    const bool ok = wait_warp(mma_bar, 0, abort_flag, status) && wait_warp(ld_bar, 0, abort_flag, status);
-    if (ok) {
-        tc_fence_after();
-        const int q = warp & 3, e = warp >> 2, row = 32 * q + lane;
-        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + 64 * e;
-        const float w = cum[e * kBlk + row];
-        unsigned char *yr = y_tile + e * kPanel;
+        if (tid == 0) {  // the MMAs of block i (the accumulator was read out by block i - 1's epilogue)
+            if (wait_phase(&ld_bar[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag, status)) {
+                tc_fence_after();
+                const uint32_t ca = smem_u32(c_tile), sa = smem_u32(s_tile);
+                constexpr uint32_t kId = idesc(128, 128, false, false);
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-            uint32_t acc[32];
-            tmem_ld32(taddr + 32 * half, acc);
-            tmem_wait_ld(acc);
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {  // 16-byte chunks 4 half + c4 of the row (8 columns each)
-                uint4 *pv = reinterpret_cast<uint4 *>(yr + swz(row, 4 * half + c4));
-                const uint4 old = *pv;
-                const uint32_t ov[4] = {old.x, old.y, old.z, old.w};
-                uint32_t nv[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float a0 = __uint_as_float(acc[8 * c4 + 2 * u]), a1 = __uint_as_float(acc[8 * c4 + 2 * u + 1]);
-                    nv[u] = pack_bf16(fmaf(w, a0, bf16_lo(ov[u])), fmaf(w, a1, bf16_hi(ov[u])));
+                for (int kk = 0; kk < N / 16; ++kk) {
+                    const uint32_t off = (uint32_t)((kk >> 2) * kPanel + (kk & 3) * 32);
+                    mma_ss(tmem, sdesc(ca + off, 16, 1024), sdesc(sa + off, 16, 1024), kId, kk > 0);
                 }
-                *pv = make_uint4(nv[0], nv[1], nv[2], nv[3]);
+                mma_commit(mma_bar);
+                last_mma = i;
             }
         }
+        ok = wait_warp(mma_bar, (uint32_t)i & 1u, abort_flag, status) &&
+             wait_warp(&ld_bar[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag, status);
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
+        tc_fence_after();
+        // C is free once the MMAs are done, and y buffer (i + 1) % 2 once the store of block i - 1
+        // has read it: the next block's tiles load during this block's epilogue
+        if (tid == 0 && i + 1 < nb) {
+            bulk_wait_read();
+            issue_loads(i + 1);
+            last_ld = i + 1;
+        }
+        {
+            const float w = cum[e * kBlk + row];
+            unsigned char *yr = y_tile + ((i & 1) * 2 + e) * kPanel;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                uint32_t acc[32];
+                tmem_ld32(taddr + 32 * half, acc);
+                tmem_wait_ld(acc);
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {  // 16-byte chunks 4 half + c4 of the row (8 columns each)
+                    uint4 *pv = reinterpret_cast<uint4 *>(yr + swz(row, 4 * half + c4));
+                    const uint4 old = *pv;
+                    const uint32_t ov[4] = {old.x, old.y, old.z, old.w};
+                    uint32_t nv[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float a0 = __uint_as_float(acc[8 * c4 + 2 * u]), a1 = __uint_as_float(acc[8 * c4 + 2 * u + 1]);
+                        nv[u] = pack_bf16(fmaf(w, a0, bf16_lo(ov[u])), fmaf(w, a1, bf16_hi(ov[u])));
+                    }
+                    *pv = make_uint4(nv[0], nv[1], nv[2], nv[3]);
+                }
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();  // y tiles written, accumulator and cum read out
+        if (tid == 0) {
+            for (int hh = 0; hh < 2; ++hh)
+                tma_store_4d(&tm_y, y_tile + ((i & 1) * 2 + hh) * kPanel, 0, h0 + hh, (int)t0, b, policy_evict_first());
+            bulk_commit();
+        }
     }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && ok && !*abort_flag) {
-        for (int e = 0; e < 2; ++e) tma_store_4d(&tm_y, y_tile + e * kPanel, 0, h0 + e, (int)t0, b, policy_evict_first());
-        bulk_commit();
-        bulk_wait_all();
-    }
+    if (tid == 0) bulk_wait_all();
     if (warp == 0) {
-        if (lane == 0 && !ok) {  // MMAs still in flight must finish before TMEM is released
+        if (lane == 0 && !ok) {  // MMAs and loads still in flight end before TMEM and the CTA go
             const unsigned long long w0 = now_ns();
-            while (!mbar_try(mma_bar, 0) && now_ns() - w0 < kWaitNs) {
+            while (last_mma >= 0 && !mbar_try(mma_bar, (uint32_t)last_mma & 1u) && now_ns() - w0 < kWaitNs) {
+            }
+            while (last_ld >= 0 && !mbar_try(&ld_bar[last_ld & 1], (uint32_t)(last_ld >> 1) & 1u) &&
+                   now_ns() - w0 < 2 * kWaitNs) {
             }
         }
         __syncwarp();
@@ -226,10 +256,15 @@ cudaError_t cp_correct_tc_launch(const CpProblem &p, const void *dt, const float
     prm.N = (int)p.N;
     prm.nblk = nblk;
     prm.pairs_per_group = (int)(p.H / p.G / 2);
+    // about one CTA per SM: each takes a run of consecutive blocks of one (batch row, head pair)
+    const long long tiles = (long long)nblk * p.G * prm.pairs_per_group * p.B;
+    const int sms = tc::num_sms() > 0 ? tc::num_sms() : 148;
+    prm.blocks_per_cta = (int)std::max(1ll, std::min((long long)nblk, (tiles + sms - 1) / sms));
     const int smem = smem_bytes((int)p.N) + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_correct_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)nblk, (unsigned)(p.G * prm.pairs_per_group), (unsigned)p.B);
+    dim3 grid((unsigned)((nblk + prm.blocks_per_cta - 1) / prm.blocks_per_cta), (unsigned)(p.G * prm.pairs_per_group),
+              (unsigned)p.B);
     k_correct_tc<<<grid, kThreads, smem, s>>>(tmc, tmy, prm);
     return cudaGetLastError();
 }
