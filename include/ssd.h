@@ -158,7 +158,9 @@ ssd_status_t ssd_fwd_static_scratch(const ssd_shape_t *shape, ssd_dtype_t dtype,
  *   states_out  [B, K, H, P, N]   fp32 or NULL   state after draft token k
  *   y           [B, K, H, P]      dtype          outputs of the K tokens
  * Requires dstate % 4 == 0. With states_out == NULL only y is written: the flow
- * that keeps one state (ssd_advance_state below) instead of all K.
+ * that keeps one state (ssd_advance_state below) instead of all K. That case evaluates
+ * the K tokens in the chunked form (each state row read once, no per-token state chain),
+ * so its y can differ from the states_out != NULL case in the last bits.
  */
 ssd_status_t ssd_verify(const ssd_shape_t *shape, ssd_dtype_t dtype, const float *h0,
                         const void *x, const void *dt, const float *A, const void *Bm,

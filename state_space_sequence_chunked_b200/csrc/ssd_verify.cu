@@ -9,7 +9,8 @@
 //
 // The same write-up notes that storing every intermediate state is what a
 // hardware-aware verify should avoid. Two kernels serve that flow without states_out:
-// verify with states_out = NULL writes only y, and k_advance recomputes, once the
+// verify with states_out = NULL writes only y (k_verify_y: the chunked form over the K tokens,
+// without the per-token state chain), and k_advance recomputes, once the
 // accepted counts are known, the state after accepted[b] tokens straight from h0
 // (K small steps per state row in registers: one read of h0 and one write of the
 // kept state). It applies the same fp32 operations in the same order as k_verify,
@@ -127,6 +128,117 @@ __global__ void __launch_bounds__(kVThreads)
             const float tot = reduce8(part, lane);
             const int k = k0 + (lane >> 2);
             if ((lane & 3) == 0 && k < K) store_as(y + (((int64_t)b * K + k) * H + h) * P + p, tot + Dh * xsm[k * P + p]);
+        }
+    }
+}
+
+// grid (H, B). Verify with outputs only: no state is written, so the K-token chunked form of the
+// same recurrence (the quadratic "SSD 层的对偶注意力" form within a chunk of K tokens, plus the
+// initial state decayed to each token) replaces the per-token state chain:
+//     y_k = exp(cum_k) (C_k . h0[p, :]) + sum_{s <= k} M[k, s] x_s[p] + D_h x_k[p],
+//     M[k, s] = (C_k . B_s) exp(cum_k - cum_s) dt_s,   cum_k = sum_{j <= k} dt_j A_h.
+// Each state row is read once and its K dot products with C are independent. M (K x K) is
+// formed once per CTA. Shared memory: B, C (K x N), x (K x P), cum, dt (K), M (K x K).
+template <typename T>
+__global__ void __launch_bounds__(kVThreads)
+    k_verify_y(const float *__restrict__ h0, const T *__restrict__ x, const T *__restrict__ dt,
+               const float *__restrict__ A, const T *__restrict__ Bm, const T *__restrict__ Cm,
+               const float *__restrict__ D, int K, int H, int P, int G, int N, T *__restrict__ y) {
+    extern __shared__ float sm[];
+    float *bsm = sm;            // [K][N]
+    float *csm = bsm + K * N;   // [K][N]
+    float *xsm = csm + K * N;   // [K][P]
+    float *dts = xsm + K * P;   // [K]
+    float *cum = dts + K;       // [K]
+    float *msm = cum + K;       // [K][K]
+    const int h = blockIdx.x, b = blockIdx.y, g = h / (H / G);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < K * N; i += blockDim.x) {
+        const int k = i / N, n = i % N;
+        const int64_t off = (((int64_t)b * K + k) * G + g) * N + n;
+        bsm[i] = to_f32(Bm[off]);
+        csm[i] = to_f32(Cm[off]);
+    }
+    for (int i = tid; i < K * P; i += blockDim.x) {
+        const int k = i / P, p = i % P;
+        xsm[i] = to_f32(x[(((int64_t)b * K + k) * H + h) * P + p]);
+    }
+    if (warp == 0) {  // dt and the inclusive cumsum of dt A (K <= 64: two tokens per lane)
+        float d[2], a[2];
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            const int k = 2 * lane + m;
+            d[m] = k < K ? to_f32(dt[((int64_t)b * K + k) * H + h]) : 0.f;
+            a[m] = d[m] * A[h];
+        }
+        a[1] += a[0];
+        float incl = a[1];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
+        }
+        const float excl = incl - a[1];
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            const int k = 2 * lane + m;
+            if (k < K) {
+                dts[k] = d[m];
+                cum[k] = excl + a[m];
+            }
+        }
+    }
+    __syncthreads();
+    // M[k, s] for s <= k (zero above the diagonal): one warp per entry, lanes over n
+    for (int e = warp; e < K * K; e += kVThreads / 32) {
+        const int k = e / K, s2 = e % K;
+        float v = 0.f;
+        if (s2 <= k) {
+            for (int n = lane; n < N; n += 32) v = fmaf(csm[k * N + n], bsm[s2 * N + n], v);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            v *= expf(cum[k] - cum[s2]) * dts[s2];
+        }
+        if (lane == 0) msm[e] = v;
+    }
+    __syncthreads();
+    const int nv = N / 4;
+    const float Dh = D ? D[h] : 0.f;
+    for (int p = warp; p < P; p += kVThreads / 32) {
+        float4 s[kMaxVec];
+        const float4 *src = reinterpret_cast<const float4 *>(h0 + (((int64_t)b * H + h) * P + p) * N);
+#pragma unroll
+        for (int j = 0; j < kMaxVec; ++j) {
+            const int v = lane + 32 * j;
+            s[j] = v < nv ? src[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        for (int k0 = 0; k0 < K; k0 += 8) {
+            float part[8];
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const int k = k0 + kk;
+                part[kk] = 0.f;
+                if (k >= K) continue;  // warp-uniform
+                const float4 *ck = reinterpret_cast<const float4 *>(csm + k * N);
+#pragma unroll
+                for (int j = 0; j < kMaxVec; ++j) {
+                    const int v = lane + 32 * j;
+                    if (v < nv) {
+                        const float4 cc = ck[v];
+                        part[kk] = fmaf(s[j].x, cc.x, part[kk]);
+                        part[kk] = fmaf(s[j].y, cc.y, part[kk]);
+                        part[kk] = fmaf(s[j].z, cc.z, part[kk]);
+                        part[kk] = fmaf(s[j].w, cc.w, part[kk]);
+                    }
+                }
+            }
+            const float tot = reduce8(part, lane);
+            const int k = k0 + (lane >> 2);
+            if ((lane & 3) == 0 && k < K) {
+                float acc = expf(cum[k]) * tot;
+                for (int s2 = 0; s2 <= k; ++s2) acc = fmaf(msm[k * K + s2], xsm[s2 * P + p], acc);
+                store_as(y + (((int64_t)b * K + k) * H + h) * P + p, acc + Dh * xsm[k * P + p]);
+            }
         }
     }
 }
@@ -286,6 +398,25 @@ __global__ void k_select(const float *__restrict__ h0, const float *__restrict__
 
 cudaError_t verify_launch(const VerifyProblem &p, cudaStream_t s) {
     const int K = (int)p.K, H = (int)p.H, P = (int)p.P, G = (int)p.G, N = (int)p.N;
+    if (!p.states_out) {  // outputs only: the chunked form, no state chain
+        const size_t smem = (size_t)(2 * K * N + K * P + 2 * K + K * K) * sizeof(float);
+        dim3 grid(H, (unsigned)p.B);
+        cudaError_t e;
+        if (p.dtype == SSD_F32) {
+            if ((e = cudaFuncSetAttribute(k_verify_y<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+                return e;
+            k_verify_y<float><<<grid, kVThreads, smem, s>>>(p.h0, (const float *)p.x, (const float *)p.dt, p.A,
+                                                            (const float *)p.Bm, (const float *)p.Cm, p.D, K, H, P, G,
+                                                            N, (float *)p.y);
+        } else {
+            using bf = __nv_bfloat16;
+            if ((e = cudaFuncSetAttribute(k_verify_y<bf>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+                return e;
+            k_verify_y<bf><<<grid, kVThreads, smem, s>>>(p.h0, (const bf *)p.x, (const bf *)p.dt, p.A, (const bf *)p.Bm,
+                                                         (const bf *)p.Cm, p.D, K, H, P, G, N, (bf *)p.y);
+        }
+        return cudaGetLastError();
+    }
     const size_t smem = (size_t)(2 * K * N + K * P + 2 * K) * sizeof(float);
     cudaError_t e;
     dim3 grid(H, (unsigned)p.B);
