@@ -33,7 +33,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("ssd_fwd", "ssd_verify", "ssd_select_state", "ssd_fwd_workspace_bytes", "ssd_strerror",
-              "ssd_advance_state", "ssd_decode_step"):
+              "ssd_advance_state", "ssd_decode_step", "ssd_cp_decay", "ssd_cp_combine", "ssd_cp_correct"):
         assert n in names
 
 
@@ -155,6 +155,39 @@ def test_advance_and_decode_reject_before_launch(lib):
     assert dec(state=None) == 1
     assert dec(y=0x5002) == 3
     assert dec(D=0x6004) == 3
+
+
+def test_context_parallel_steps_reject_before_launch(lib):
+    vp = lambda a: ctypes.c_void_p(a) if a else None
+    s = B.ShapeT(2, 300, 4, 64, 1, 128)
+
+    def decay(shape=s, dtype=1, dt=0x1000, A=0x2000, bd=0x3000, tot=0x4000):
+        return lib.ssd_cp_decay(ctypes.byref(shape), dtype, vp(dt), vp(A), vp(bd), vp(tot), None)
+
+    assert decay(dtype=7) == 1
+    assert decay(tot=None) == 1
+    assert decay(dt=None) == 1                                   # L > 0 needs dt and block sums
+    assert decay(A=0x2004) == 3
+    assert decay(shape=B.ShapeT(2, 300, 4, 64, 3, 128)) == 1    # heads not a multiple of groups
+    assert decay(shape=B.ShapeT(0, 300, 4, 64, 1, 128), dt=None, A=None, bd=None, tot=None) == 0
+
+    def combine(shape=s, R=4, rank=1, states=0x1000, totals=0x2000, s_in=0x3000, hf=0x4000):
+        return lib.ssd_cp_combine(ctypes.byref(shape), R, rank, vp(states), vp(totals), vp(s_in), vp(hf), None)
+
+    assert combine(R=0) == 1 and combine(rank=4) == 1 and combine(rank=-1) == 1
+    assert combine(R=70000, rank=0) == 2
+    assert combine(s_in=None) == 1
+    assert combine(hf=0x4008) == 3
+    assert combine(shape=B.ShapeT(2, 300, 4, 1, 1, 3)) == 2       # headdim * dstate % 4
+
+    def correct(shape=s, dt=0x1000, y=0x5000, status=None):
+        return lib.ssd_cp_correct(ctypes.byref(shape), 1, vp(dt), vp(0x2000), vp(0x3000), vp(0x4000), vp(0x6000),
+                                  vp(y), vp(status), None)
+
+    assert correct(dt=None) == 1
+    assert correct(y=0x5008) == 3
+    assert correct(status=0x7002) == 3                           # the status word is an int32
+    assert correct(shape=B.ShapeT(2, 0, 4, 64, 1, 128), dt=None) == 0   # empty segment: nothing to do
 
 
 def test_binding_requires_cuda_tensors():
