@@ -24,6 +24,12 @@ Forms (each in fp64 on the already-rounded inputs, layouts as in the library):
                      state after every token; select_state keeps the state at the
                      accepted position: "distilling Llama into Mamba" write-up,
                      "推测解码".
+  backward           the gradient of sum(dy * y) + sum(dh_final * h_final) with
+                     respect to every input: the recurrence differentiated token
+                     by token in reverse (C, OpenMP over (b, h)); the states are
+                     recomputed per segment in the reverse sweep instead of being
+                     stored, as "A Visual Guide to Mamba and SSMs",
+                     "Recomputation", describes for the backward pass.
 Layouts: x [B,L,H,P], dt [B,L,H], A [H], Bm/Cm [B,L,G,N], D [H], h0 [B,H,P,N];
 head h uses group g = h // (H // G).
 """
@@ -47,6 +53,8 @@ def _load():
         i64, dp = ctypes.c_int64, ctypes.POINTER(ctypes.c_double)
         lib.oracle_ssd_recurrent.argtypes = [i64] * 6 + [dp] * 10 + [ctypes.c_int]
         lib.oracle_ssd_recurrent.restype = ctypes.c_int
+        lib.oracle_ssd_backward.argtypes = [i64] * 6 + [dp] * 9 + [dp] * 7 + [i64, ctypes.c_int]
+        lib.oracle_ssd_backward.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -77,6 +85,29 @@ def recurrent(x, dt, A, Bm, Cm, D=None, h0=None, *, store_states=False, threads=
     if rc != 0:
         raise RuntimeError("oracle_ssd_recurrent failed")
     return (y, hf, st) if store_states else (y, hf)
+
+
+def backward(x, dt, A, Bm, Cm, D, h0, dy, dh_final=None, *, seg=64, threads=0):
+    """Gradient of sum(dy * y) + sum(dh_final * h_final) through the recurrence.
+
+    D and h0 may be None (no skip / zero initial state), dh_final None (= 0).
+    Returns a dict: dx [B,L,H,P], ddt [B,L,H], dA [H], dB [B,L,G,N], dC [B,L,G,N],
+    dD [H], dh0 [B,H,P,N] (the gradient for the initial state, also when h0 is None)."""
+    x, dt, A, Bm, Cm, D, h0, dy, dh_final = map(_f64, (x, dt, A, Bm, Cm, D, h0, dy, dh_final))
+    Bsz, L, H, P = x.shape
+    G, N = Bm.shape[2], Bm.shape[3]
+    assert dt.shape == (Bsz, L, H) and A.shape == (H,) and Bm.shape == Cm.shape == (Bsz, L, G, N)
+    assert dy.shape == x.shape and H % G == 0
+    out = {"dx": np.empty_like(x), "ddt": np.empty_like(dt), "dA": np.empty(H),
+           "dB": np.empty_like(Bm), "dC": np.empty_like(Cm), "dD": np.empty(H),
+           "dh0": np.empty((Bsz, H, P, N))}
+    rc = _load().oracle_ssd_backward(
+        Bsz, L, H, P, G, N, _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D), _ptr(h0),
+        _ptr(dy), _ptr(dh_final), _ptr(out["dx"]), _ptr(out["ddt"]), _ptr(out["dA"]),
+        _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dh0"]), int(seg), int(threads))
+    if rc != 0:
+        raise RuntimeError("oracle_ssd_backward failed")
+    return out
 
 
 def _heads_to_groups(Bm, H):
