@@ -189,10 +189,11 @@ def barrier(ws):
 # ---------------------------------------------------------------------------------------
 # CPU oracle timing (the CPU baseline and the reference arm)
 
-def time_oracle(wl, d, target_s: float):
+def time_oracle(wl, d, target_s: float, backward=None):
     """Run the fp64 oracle on whole (b, h) streams (every token of the sequence) of
     the drawn inputs, as many streams as fit in about target_s. Returns (tokens/s
-    extrapolated to the whole problem, streams run, threads, seconds)."""
+    extrapolated to the whole problem, streams run, threads, seconds). With `backward`
+    (the drawn cotangents) it times the oracle's backward pass instead."""
     import oracle
 
     threads = os.cpu_count() or 1
@@ -210,7 +211,12 @@ def time_oracle(wl, d, target_s: float):
         A, D = d["A"].value[:nh], d["D"].value[:nh]
         h0 = d["h0"].values((slice(0, nb), slice(0, nh))) if d["h0"] is not None else None
         t0 = time.perf_counter()
-        oracle.recurrent(x, dt, A, Bm, Cm, D, h0, threads=threads)
+        if backward is None:
+            oracle.recurrent(x, dt, A, Bm, Cm, D, h0, threads=threads)
+        else:
+            dy = backward["dy"].values(hs)
+            dhf = backward["dh_final"].values((slice(0, nb), slice(0, nh))) if backward["dh_final"] else None
+            oracle.backward(x, dt, A, Bm, Cm, D, h0, dy, dhf, threads=threads)
         return time.perf_counter() - t0, nb * nh
 
     t1, n1 = run(1, 1)
@@ -338,6 +344,154 @@ def verify_main(args, wl):
     return 0
 
 
+BWD_METRIC = "SSD bwd tokens/s (batch·seqlen/s) at 2.7B-layer shape; % of roofline"
+
+
+def bwd_algorithmic(wl):
+    """FLOPs of the chunked backward with recomputation (causal pairs only, C B^T once per
+    (batch, chunk, group), each dot product dy.x counted once) and the bytes of its inputs
+    read once and gradients written once."""
+    B, L, H, P, N, G, Q = wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.dstate, wl.ngroups, wl.chunk
+    e = 2 if wl.dtype == "bf16" else 4
+    nc_full, tail = divmod(L, Q)
+    tri = lambda q: q * (q + 1) / 2
+    pairs = nc_full * tri(Q) + tri(tail)
+    # per head: dy.x, u (P wide), v and w (N wide) over the pairs; five P x N products per
+    # token (recomputed chunk state, adjoint chunk sum, Gend B, Gend^T x, S_in^T dy)
+    flops = B * (2 * pairs * N * G + H * pairs * (4 * P + 4 * N)) + 10 * B * L * H * P * N
+    nbytes = (3 * B * L * H * P * e          # x, dy in; dx out
+              + 2 * B * L * H * e            # dt in; ddt out
+              + 4 * B * L * G * N * e        # B, C in; dB, dC out
+              + 4 * H * 4                    # A, D in; dA, dD out
+              + 2 * B * H * P * N * 4        # dh_final in; dh0 out
+              + (B * H * P * N * 4 if wl.h0_std > 0 else 0))
+    return nbytes, flops
+
+
+def alu_peak_tflops(clock_mhz):
+    """fp32 FMA peak of the CUDA cores: 148 SMs x 128 fp32 lanes x 2 FLOP per clock."""
+    return 148 * 128 * 2 * clock_mhz * 1e6 / 1e12
+
+
+def bwd_main(args, wl):
+    """One step = one ssd_bwd call (gradients of every input, states recomputed) on seeded
+    inputs and cotangents resident in HBM."""
+    import torch
+
+    from state_space_sequence_chunked_b200 import _binding as ssd
+    from state_space_sequence_chunked_b200 import inputs
+
+    ws, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    d = inputs.draw(wl, seed=rank_seed(wl, rank))
+    cot = inputs.draw_cotangents(wl, seed=rank_seed(wl, rank))
+    code = ssd.SSD_BF16 if wl.dtype == "bf16" else ssd.SSD_F32
+    g = {k: d[k].torch(dev) for k in ("x", "dt", "A", "B", "C", "D")}
+    g["dy"] = cot["dy"].torch(dev)
+    g["dhf"] = cot["dh_final"].torch(dev)
+    h0 = d["h0"].torch(dev) if d["h0"] is not None else None
+    need = ssd.bwd_workspace_bytes(wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.ngroups, wl.dstate, code,
+                                   wl.chunk)
+    work = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    out = {"dx": torch.empty_like(g["x"]), "ddt": torch.empty_like(g["dt"]), "dA": torch.empty_like(g["A"]),
+           "dB": torch.empty_like(g["B"]), "dC": torch.empty_like(g["C"]), "dD": torch.empty_like(g["D"]),
+           "dh0": torch.empty_like(g["dhf"])}
+    stream = torch.cuda.current_stream(dev)
+    launches = 11
+
+    def call(src):
+        ssd.ssd_bwd(src["x"], src["dt"], src["A"], src["B"], src["C"], src["D"], h0, src["dy"], src["dhf"],
+                    chunk=wl.chunk, out=out, workspace=work, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        call(g)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev)
+    clocks.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    clocks.mark_start()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        call(g)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark_end()
+    barrier(ws)
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms_max = reduce_max(ms, ws)
+
+    # end to end: inputs and cotangents from pinned host memory, every gradient back
+    host = {k: v.cpu().pin_memory() for k, v in g.items()}
+    dg = {k: torch.empty_like(v) for k, v in g.items()}
+    out_host = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in out.items()}
+
+    def e2e_step():
+        for k in dg:
+            dg[k].copy_(host[k], non_blocking=True)
+        call(dg)
+        for k in out:
+            out_host[k].copy_(out[k], non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 5))
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    e2e_ms = reduce_max(ev0.elapsed_time(ev1) / e2e_steps, ws)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(v.numel() * v.element_size() for v in out_host.values())
+
+    tokens = wl.batch * wl.seqlen
+    nbytes, flops = bwd_algorithmic(wl)
+    hbm, tf, src = peaks()
+    clk_mhz = clk.get("sm_mhz") or 1965.0
+    alu = alu_peak_tflops(clk.get("sm_max_mhz") or 1965.0)
+    achieved = flops / (ms * 1e-3) / 1e12
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        v, n, threads, t = time_oracle(wl, d, args.cpu_seconds, backward=cot)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"fp64 backward of the recurrence on {n} of {wl.batch * wl.nheads} (batch, head) streams "
+                         f"over all {wl.seqlen} tokens ({t:.1f} s), extrapolated to the whole batch"}
+    if rank == 0:
+        line = {
+            "metric": BWD_METRIC, "value": tokens * ws / (ms_max * 1e-3), "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name + " backward", "batch": wl.batch, "seqlen": wl.seqlen,
+                       "nheads": wl.nheads, "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups,
+                       "chunk": wl.chunk, "io_dtype": wl.dtype,
+                       "l2": "inputs larger than L2 (x, dy, dx 335.5 MB each per step vs 126 MB L2); no flush"},
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": alu, "unit": "TFLOP/s",
+                         "frac": achieved / alu, "traffic": None,
+                         "kernel": "whole ssd_bwd call (%d launches, fp32 FMA on CUDA cores)" % launches,
+                         "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x max SM clock",
+                         "alg_flops": flops, "alg_bytes": nbytes,
+                         "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / hbm,
+                         "tensor_roofline_ms": flops / (tf * 1e12) * 1e3,
+                         "hbm_roofline_ms": nbytes / (hbm * 1e9) * 1e3, "sm_mhz_median": clk_mhz},
+            "cpu_baseline": cpu,
+            "e2e": {"value": tokens * ws / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches * args.steps, "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
 def aux_main(args):
     """Per-kernel timings of the kernels beside the forward, each against the HBM roofline
     (all of them are bandwidth-bound): the two verify flows on the spec-decode workload
@@ -444,6 +598,8 @@ def main():
     ap.add_argument("--workload", default="mamba2_2p7b")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the backward pass (ssd_bwd) of the forward workload instead")
     ap.add_argument("--aux", action="store_true",
                     help="time the verify/decode and context-parallel kernels instead (1 GPU, one line per kernel)")
     args = ap.parse_args()
@@ -453,6 +609,10 @@ def main():
     from state_space_sequence_chunked_b200 import inputs
 
     wl = inputs.WORKLOADS[args.workload]
+    if args.bwd:
+        if args.impl == "reference" or wl.verify:
+            raise SystemExit("--bwd times this library's backward of a forward workload")
+        return bwd_main(args, wl)
     if wl.verify:
         if args.impl == "reference":
             raise SystemExit("the reference arm times the forward workloads")

@@ -274,6 +274,37 @@ ssd_status_t ssd_cp_correct(const ssd_shape_t *shape, ssd_dtype_t dtype, const v
                             const void *Cm, const float *block_decay, const float *s_in, void *y,
                             int32_t *status, void *stream);
 
+/*
+ * Backward pass of ssd_fwd: given the cotangents dy of y and dh_final of h_final, the
+ * gradient of  sum(dy * y) + sum(dh_final * h_final)  with respect to every input.
+ * The states are recomputed from the inputs rather than stored by the forward (the
+ * recomputation of the hardware-aware algorithm, "A Visual Guide to Mamba and SSMs",
+ * section "Recomputation"); the chunks follow "SSD 算法：分块和状态传递" of the SSD
+ * write-up, run in reverse.
+ *   x, dt, A, Bm, Cm, D, h0, chunk   the forward's inputs, as in ssd_fwd
+ *   dy        [B, L, H, P]   dtype          cotangent of y
+ *   dh_final  [B, H, P, N]   fp32 or NULL   cotangent of h_final (NULL = 0)
+ *   dx        [B, L, H, P]   dtype          out
+ *   ddt       [B, L, H]      dtype          out
+ *   dA        [H]            fp32           out (summed over the batch)
+ *   dBm, dCm  [B, L, G, N]   dtype          out (summed over the heads of each group)
+ *   dD        [H]            fp32 or NULL   out (also when D is NULL: the gradient at D = 0)
+ *   dh0       [B, H, P, N]   fp32 or NULL   out (also when h0 is NULL: the gradient at h0 = 0)
+ *   workspace, workspace_bytes              >= ssd_bwd_workspace_bytes(...)
+ * Arithmetic is fp32 on CUDA cores for both dtypes. dBm and dCm are summed with fp32
+ * atomics, so their last bits can differ between runs. batch == 0 zeroes dA and dD;
+ * seqlen == 0 also writes dh0 = dh_final (or zeros).
+ * Errors as ssd_fwd; SSD_ERR_UNSUPPORTED when headdim and dstate are too large for the
+ * kernels' shared-memory tiles together (never for headdim, dstate <= 256).
+ */
+ssd_status_t ssd_bwd_workspace_bytes(const ssd_shape_t *shape, ssd_dtype_t dtype, int64_t chunk,
+                                     size_t *bytes);
+ssd_status_t ssd_bwd(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *x, const void *dt,
+                     const float *A, const void *Bm, const void *Cm, const float *D, const float *h0,
+                     int64_t chunk, const void *dy, const float *dh_final, void *dx, void *ddt,
+                     float *dA, void *dBm, void *dCm, float *dD, float *dh0, void *workspace,
+                     size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -50,6 +50,9 @@ _SIGS = {
     "ssd_cp_decay": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 5, ctypes.c_int),
     "ssd_cp_combine": ([ctypes.POINTER(ShapeT), _i64, _i64] + [_vp] * 5, ctypes.c_int),
     "ssd_cp_correct": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 8, ctypes.c_int),
+    "ssd_bwd_workspace_bytes": ([ctypes.POINTER(ShapeT), ctypes.c_int, _i64, ctypes.POINTER(_sz)], ctypes.c_int),
+    "ssd_bwd": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 7 + [_i64] + [_vp] * 9 + [_vp, _sz, _vp],
+                ctypes.c_int),
 }
 
 CP_BLOCK = 128  # SSD_CP_BLOCK: tokens per decay block
@@ -254,3 +257,42 @@ def ssd_cp_correct(dt, A, C, block_decay, s_in, y, *, status=None, stream=None):
                               _ptr(s_in), _ptr(y), _ptr(status), _stream(dev, stream))
     _check(st, "ssd_cp_correct")
     return y
+
+
+def bwd_workspace_bytes(batch, seqlen, nheads, headdim, ngroups, dstate, dtype_code, chunk) -> int:
+    shape = ShapeT(batch, seqlen, nheads, headdim, ngroups, dstate)
+    out = _sz(0)
+    _check(lib().ssd_bwd_workspace_bytes(ctypes.byref(shape), dtype_code, chunk, ctypes.byref(out)),
+           "ssd_bwd_workspace_bytes")
+    return out.value
+
+
+def ssd_bwd(x, dt, A, B, C, D, h0, dy, dh_final=None, *, chunk: int, want_dD: bool = True,
+            want_dh0: bool = True, out=None, workspace=None, stream=None):
+    """Gradients of sum(dy * y) + sum(dh_final * h_final) through ssd_fwd.
+
+    Returns a dict dx, ddt, dA, dB, dC, dD (None unless want_dD), dh0 (None unless want_dh0);
+    `out` may supply any of those tensors to write into."""
+    dev = _dev(x, dt, A, B, C, D, h0, dy, dh_final, workspace)
+    Bsz, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    code = _dtype_code(x)
+    shape = ShapeT(Bsz, L, H, P, G, N)
+    o = dict(out or {})
+    o.setdefault("dx", torch.empty_like(x))
+    o.setdefault("ddt", torch.empty_like(dt))
+    o.setdefault("dA", torch.empty(H, dtype=torch.float32, device=dev))
+    o.setdefault("dB", torch.empty_like(B))
+    o.setdefault("dC", torch.empty_like(C))
+    o.setdefault("dD", torch.empty(H, dtype=torch.float32, device=dev) if want_dD else None)
+    o.setdefault("dh0", torch.empty((Bsz, H, P, N), dtype=torch.float32, device=dev) if want_dh0 else None)
+    need = bwd_workspace_bytes(Bsz, L, H, P, G, N, code, chunk)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().ssd_bwd(ctypes.byref(shape), code, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                       _ptr(h0), chunk, _ptr(dy), _ptr(dh_final), _ptr(o["dx"]), _ptr(o["ddt"]), _ptr(o["dA"]),
+                       _ptr(o["dB"]), _ptr(o["dC"]), _ptr(o["dD"]), _ptr(o["dh0"]), _ptr(workspace), ws_bytes,
+                       _stream(dev, stream))
+    _check(st, "ssd_bwd")
+    return o

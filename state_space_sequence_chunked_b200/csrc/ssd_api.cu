@@ -272,3 +272,55 @@ SSD_API ssd_status_t ssd_cp_correct(const ssd_shape_t *shape, ssd_dtype_t dtype,
     return from_cuda(cp_correct_launch(make_cp(shape, dtype), dt, A, Cm, block_decay, s_in, y, status,
                                        static_cast<cudaStream_t>(stream)));
 }
+
+SSD_API ssd_status_t ssd_bwd_workspace_bytes(const ssd_shape_t *shape, ssd_dtype_t dtype, int64_t chunk,
+                                             size_t *bytes) {
+    if (!bytes) return SSD_ERR_INVALID_ARG;
+    FwdProblem p;
+    const ssd_status_t st = make_fwd(shape, dtype, chunk, &p);
+    if (st != SSD_OK) return st;
+    if (!simt_bwd_supported(p)) return SSD_ERR_UNSUPPORTED;
+    *bytes = (p.B == 0 || p.L == 0) ? 0 : simt_bwd_workspace_bytes(p);
+    return SSD_OK;
+}
+
+SSD_API ssd_status_t ssd_bwd(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *x, const void *dt,
+                             const float *A, const void *Bm, const void *Cm, const float *D,
+                             const float *h0, int64_t chunk, const void *dy, const float *dh_final,
+                             void *dx, void *ddt, float *dA, void *dBm, void *dCm, float *dD, float *dh0,
+                             void *workspace, size_t workspace_bytes, void *stream) {
+    FwdProblem p;
+    ssd_status_t st = make_fwd(shape, dtype, chunk, &p);
+    if (st != SSD_OK) return st;
+    if (!simt_bwd_supported(p)) return SSD_ERR_UNSUPPORTED;
+    if (!dA) return SSD_ERR_INVALID_ARG;
+    const void *small[] = {dA, dD, dh0, dh_final};
+    for (const void *q : small)
+        if (q && !aligned16(q)) return SSD_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t head_bytes = (size_t)p.H * sizeof(float);
+    if (p.B == 0 || p.L == 0) {
+        cudaError_t e = cudaMemsetAsync(dA, 0, head_bytes, s);
+        if (!e && dD) e = cudaMemsetAsync(dD, 0, head_bytes, s);
+        if (!e && dh0 && p.B > 0) {
+            const size_t state_bytes = (size_t)(p.B * p.H * p.P * p.N) * sizeof(float);
+            e = dh_final ? cudaMemcpyAsync(dh0, dh_final, state_bytes, cudaMemcpyDeviceToDevice, s)
+                         : cudaMemsetAsync(dh0, 0, state_bytes, s);
+        }
+        return from_cuda(e);
+    }
+    if (!x || !dt || !A || !Bm || !Cm || !dy || !dx || !ddt || !dBm || !dCm) return SSD_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, dt, A, Bm, Cm, D, h0, dy, dx, ddt, dBm, dCm, workspace};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return SSD_ERR_ALIGNMENT;
+    if (!workspace || workspace_bytes < simt_bwd_workspace_bytes(p)) return SSD_ERR_WORKSPACE;
+    p.x = x;
+    p.dt = dt;
+    p.A = A;
+    p.Bm = Bm;
+    p.Cm = Cm;
+    p.D = D;
+    p.h0 = h0;
+    const BwdGrads g{dy, dh_final, dx, ddt, dBm, dCm, dA, dD, dh0};
+    return from_cuda(simt_bwd(p, g, workspace, s));
+}

@@ -29,6 +29,14 @@ struct VerifyProblem {
     void *y;
 };
 
+// Cotangents in and gradients out of the backward pass (dh_final, dD, dh0 may be NULL).
+struct BwdGrads {
+    const void *dy;
+    const float *dh_final;
+    void *dx, *ddt, *dBm, *dCm;
+    float *dA, *dD, *dh0;
+};
+
 // A sequence segment for the context-parallel steps (ssd_cp_*).
 struct CpProblem {
     int64_t B, L, H, P, G, N;
@@ -41,6 +49,17 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // ---- chunked path with fp32 CUDA-core arithmetic (exact path for fp32 inputs) ----
 size_t simt_fwd_workspace_bytes(const FwdProblem &p);
 cudaError_t simt_fwd(const FwdProblem &p, void *ws, cudaStream_t s);
+// steps 0, 2, 3 alone: A_cs [B,H,nc,Q], dt [B,H,nc,Q], entering states [B,H,nc,P,N], h_final
+cudaError_t simt_states(const FwdProblem &p, float *acs, float *dtw, float *states, float *h_final,
+                        cudaStream_t s);
+// out[b,h,c] = sum_{l in c} exp(A_cs[l]) dy_l C_l^T   (dy [B,L,H,P] in the input dtype)
+cudaError_t simt_adjoint_chunk_sums(const FwdProblem &p, const void *dy, const float *acs, float *out,
+                                    cudaStream_t s);
+
+// ---- backward pass (chunked, states recomputed, fp32 CUDA-core arithmetic) ----------
+bool simt_bwd_supported(const FwdProblem &p);
+size_t simt_bwd_workspace_bytes(const FwdProblem &p);
+cudaError_t simt_bwd(const FwdProblem &p, const BwdGrads &g, void *ws, cudaStream_t s);
 
 // ---- fused chunked path on tcgen05 tensor cores (bf16, P = 64, N in {128, 256}) ----
 bool tc_supported(const FwdProblem &p);

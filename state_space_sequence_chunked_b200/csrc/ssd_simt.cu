@@ -11,6 +11,10 @@
 //                  exp(A_cs) C S_in^T plus the D skip
 // Workspace (fp32): A_cs [B,H,nc,Q], dt [B,H,nc,Q] (zero past the sequence end),
 // states [B,H,nc,P,N] (chunk states, overwritten in place by the entering states).
+//
+// The backward pass recomputes steps 0, 2 and 3 with these kernels (simt_states),
+// and k_chunk_state's adjoint form gives the per-chunk sums exp(A_cs[l]) dy_l C_l^T
+// that its reverse state pass consumes (simt_adjoint_chunk_sums).
 #include "ssd_internal.cuh"
 
 namespace ssd {
@@ -78,11 +82,14 @@ __global__ void __launch_bounds__(kThreads) k_cumsum(const T *__restrict__ dt,
 }
 
 // step 2. grid (nc * ntile, H, B); every thread owns 16 of the P*N outputs of its tile.
+// Forward: sum_l exp(A_cs[Q-1] - A_cs[l]) dt_l x_l B_l^T (u = x, v = B).
+// Adjoint (kAdj): sum_l exp(A_cs[l]) dy_l C_l^T (u = dy [B,L,H,P], v = C [B,L,G,N]),
+// the gradient of the chunk's state-to-output term with respect to its entering state.
 constexpr int kStateTileL = 32;
 constexpr int kStatePerThread = 16;
 constexpr int kStateTile = kThreads * kStatePerThread;
 
-template <typename T>
+template <typename T, bool kAdj>
 __global__ void __launch_bounds__(kThreads)
     k_chunk_state(const T *__restrict__ x, const T *__restrict__ Bm, const float *__restrict__ acs,
                   const float *__restrict__ dtw, int64_t L, int H, int P, int G, int N, int Q, int nc,
@@ -111,7 +118,8 @@ __global__ void __launch_bounds__(kThreads)
     for (int l0 = 0; l0 < q; l0 += kStateTileL) {
         const int nl = min(kStateTileL, q - l0);
         for (int i = threadIdx.x; i < kStateTileL; i += blockDim.x)
-            ws[i] = i < nl ? expf(last - acs[lb + l0 + i]) * dtw[lb + l0 + i] : 0.f;
+            ws[i] = i < nl ? (kAdj ? expf(acs[lb + l0 + i]) : expf(last - acs[lb + l0 + i]) * dtw[lb + l0 + i])
+                           : 0.f;
         __syncthreads();
         for (int i = threadIdx.x; i < kStateTileL * P; i += blockDim.x) {
             const int l = i / P, p = i % P;
@@ -274,37 +282,53 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-template <typename T>
-cudaError_t run(const FwdProblem &p, void *ws, cudaStream_t s) {
-    const WsLayout w = carve(p, ws);
+template <typename T, bool kAdj>
+cudaError_t launch_chunk_state(const FwdProblem &p, const void *u, const void *v, const float *acs,
+                               const float *dtw, float *out, cudaStream_t s) {
     const int H = (int)p.H, P = (int)p.P, G = (int)p.G, N = (int)p.N, Q = (int)p.Q, nc = (int)p.nc;
-    const T *x = static_cast<const T *>(p.x), *dt = static_cast<const T *>(p.dt);
-    const T *Bm = static_cast<const T *>(p.Bm), *Cm = static_cast<const T *>(p.Cm);
+    const int ntile = (P * N + kStateTile - 1) / kStateTile;
+    const size_t smem = (size_t)(kStateTileL * (P + N) + kStateTileL) * sizeof(float);
     cudaError_t e;
+    if ((e = cudaFuncSetAttribute(k_chunk_state<T, kAdj>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+        return e;
+    dim3 grid(nc * ntile, H, (unsigned)p.B);
+    k_chunk_state<T, kAdj><<<grid, kThreads, smem, s>>>(static_cast<const T *>(u), static_cast<const T *>(v), acs,
+                                                        dtw, p.L, H, P, G, N, Q, nc, ntile, out);
+    return cudaGetLastError();
+}
 
+// steps 0, 2, 3: A_cs and dt per chunk, then the state entering every chunk (in `states`)
+template <typename T>
+cudaError_t run_states(const FwdProblem &p, float *acs, float *dtw, float *states, float *h_final,
+                       cudaStream_t s) {
+    const int H = (int)p.H, P = (int)p.P, N = (int)p.N, Q = (int)p.Q, nc = (int)p.nc;
+    const T *dt = static_cast<const T *>(p.dt);
+    cudaError_t e;
     {
         const size_t smem = (size_t)Q * 33 * sizeof(float);
         if ((e = cudaFuncSetAttribute(k_cumsum<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
             return e;
         dim3 grid(nc, (H + 31) / 32, (unsigned)p.B);
-        k_cumsum<T><<<grid, kThreads, smem, s>>>(dt, p.A, p.L, H, Q, nc, w.acs, w.dtw);
+        k_cumsum<T><<<grid, kThreads, smem, s>>>(dt, p.A, p.L, H, Q, nc, acs, dtw);
         if ((e = cudaGetLastError())) return e;
     }
-    {
-        const int ntile = (P * N + kStateTile - 1) / kStateTile;
-        const size_t smem = (size_t)(kStateTileL * (P + N) + kStateTileL) * sizeof(float);
-        if ((e = cudaFuncSetAttribute(k_chunk_state<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
-            return e;
-        dim3 grid(nc * ntile, H, (unsigned)p.B);
-        k_chunk_state<T><<<grid, kThreads, smem, s>>>(x, Bm, w.acs, w.dtw, p.L, H, P, G, N, Q, nc, ntile,
-                                                      w.states);
-        if ((e = cudaGetLastError())) return e;
-    }
+    if ((e = launch_chunk_state<T, false>(p, p.x, p.Bm, acs, dtw, states, s))) return e;
     {
         dim3 grid((P * N + kThreads - 1) / kThreads, H, (unsigned)p.B);
-        k_state_pass<<<grid, kThreads, 0, s>>>(w.acs, p.h0, H, P * N, Q, nc, w.states, p.h_final);
+        k_state_pass<<<grid, kThreads, 0, s>>>(acs, p.h0, H, P * N, Q, nc, states, h_final);
         if ((e = cudaGetLastError())) return e;
     }
+    return cudaSuccess;
+}
+
+template <typename T>
+cudaError_t run(const FwdProblem &p, void *ws, cudaStream_t s) {
+    const WsLayout w = carve(p, ws);
+    const int H = (int)p.H, P = (int)p.P, G = (int)p.G, N = (int)p.N, Q = (int)p.Q, nc = (int)p.nc;
+    const T *x = static_cast<const T *>(p.x);
+    const T *Bm = static_cast<const T *>(p.Bm), *Cm = static_cast<const T *>(p.Cm);
+    cudaError_t e;
+    if ((e = run_states<T>(p, w.acs, w.dtw, w.states, p.h_final, s))) return e;
     {
         const int nrt = (Q + kRows - 1) / kRows;
         const size_t smem =
@@ -329,6 +353,18 @@ size_t simt_fwd_workspace_bytes(const FwdProblem &p) {
 
 cudaError_t simt_fwd(const FwdProblem &p, void *ws, cudaStream_t s) {
     return p.dtype == SSD_F32 ? run<float>(p, ws, s) : run<__nv_bfloat16>(p, ws, s);
+}
+
+cudaError_t simt_states(const FwdProblem &p, float *acs, float *dtw, float *states, float *h_final,
+                        cudaStream_t s) {
+    return p.dtype == SSD_F32 ? run_states<float>(p, acs, dtw, states, h_final, s)
+                              : run_states<__nv_bfloat16>(p, acs, dtw, states, h_final, s);
+}
+
+cudaError_t simt_adjoint_chunk_sums(const FwdProblem &p, const void *dy, const float *acs, float *out,
+                                    cudaStream_t s) {
+    return p.dtype == SSD_F32 ? launch_chunk_state<float, true>(p, dy, p.Cm, acs, nullptr, out, s)
+                              : launch_chunk_state<__nv_bfloat16, true>(p, dy, p.Cm, acs, nullptr, out, s);
 }
 
 }  // namespace ssd

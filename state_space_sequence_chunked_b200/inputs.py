@@ -142,3 +142,16 @@ def draw(wl: Workload, *, batch=None, seqlen=None, seed=None, h0_std=None, zero_
     if wl.verify:
         out["accepted"] = rng.integers(0, L + 1, size=(Bsz,), dtype=np.int64).astype(np.int32)
     return out
+
+
+def draw_cotangents(wl: Workload, *, batch=None, seqlen=None, seed=None, dh_std=1.0):
+    """Cotangents for the backward pass of workload `wl`: dy ~ N(0, 1) [B,L,H,P] in the
+    storage dtype and dh_final ~ N(0, dh_std) [B,H,P,N] fp32 (None when dh_std is 0).
+    Drawn from their own stream (seed + 10007), so the forward inputs are unchanged."""
+    Bsz = wl.batch if batch is None else batch
+    L = wl.seqlen if seqlen is None else seqlen
+    H, P, N = wl.nheads, wl.headdim, wl.dstate
+    rng = np.random.default_rng((wl.seed if seed is None else seed) + 10007)
+    dy = rng.standard_normal((Bsz, L, H, P))
+    dhf = rng.standard_normal((Bsz, H, P, N)) * dh_std if dh_std > 0 else None
+    return {"dy": Tensor(dy, wl.dtype), "dh_final": Tensor(dhf, "f32") if dhf is not None else None}

@@ -89,3 +89,33 @@ def sample_streams(Bsz, H, n, seed=123):
 
 def draw(name, **kw):
     return inputs.draw(inputs.WORKLOADS[name], **kw)
+
+
+GRADS = ("dx", "ddt", "dA", "dB", "dC", "dD", "dh0")
+
+
+def run_bwd(d, cot, chunk, device, *, use_D=True, use_h0=True, use_dhf=True):
+    """ssd_bwd through the binding, outputs pre-filled with NaN; returns numpy fp64 arrays."""
+    g = gpu_inputs(d, device)
+    dy = cot["dy"].torch(device)
+    dhf = cot["dh_final"].torch(device) if (use_dhf and cot["dh_final"] is not None) else None
+    out = {"dx": torch.full_like(g["x"], float("nan")), "ddt": torch.full_like(g["dt"], float("nan")),
+           "dB": torch.full_like(g["B"], float("nan")), "dC": torch.full_like(g["C"], float("nan")),
+           "dA": torch.full_like(g["A"], float("nan")), "dD": torch.full_like(g["D"], float("nan")),
+           "dh0": torch.full((g["x"].shape[0], g["x"].shape[2], g["x"].shape[3], g["B"].shape[3]), float("nan"),
+                             device=device)}
+    ssd.ssd_bwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"] if use_D else None,
+                g["h0"] if use_h0 else None, dy, dhf, chunk=chunk, out=out)
+    torch.cuda.synchronize()
+    return {k: to_np(v) for k, v in out.items()}
+
+
+def oracle_bwd(d, cot, *, use_D=True, use_h0=True, use_dhf=True, batch_rows=None):
+    """The oracle's gradients; batch_rows=(lo, hi) restricts it to those rows (dA and dD then
+    cover only them)."""
+    sl = slice(None) if batch_rows is None else slice(*batch_rows)
+    v = lambda t: t.values((sl,)) if t is not None else None
+    h0 = v(d["h0"]) if use_h0 else None
+    dhf = v(cot["dh_final"]) if use_dhf else None
+    return oracle.backward(v(d["x"]), v(d["dt"]), d["A"].value, v(d["B"]), v(d["C"]),
+                           d["D"].value if use_D else None, h0, v(cot["dy"]), dhf)

@@ -33,7 +33,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("ssd_fwd", "ssd_verify", "ssd_select_state", "ssd_fwd_workspace_bytes", "ssd_strerror",
-              "ssd_advance_state", "ssd_decode_step", "ssd_cp_decay", "ssd_cp_combine", "ssd_cp_correct"):
+              "ssd_advance_state", "ssd_decode_step", "ssd_cp_decay", "ssd_cp_combine", "ssd_cp_correct",
+              "ssd_bwd", "ssd_bwd_workspace_bytes"):
         assert n in names
 
 
@@ -109,6 +110,49 @@ def test_fwd_rejects_before_launch(lib):
     assert fwd_call(shape, GOOD, dtype=3) == 1
     # batch == 0 is a valid empty problem: nothing to launch, nothing touched
     assert fwd_call((0, 100, 4, 16, 1, 16), {k: None for k in GOOD}) == 0
+
+
+BWD_GOOD = dict(x=0x10000, dt=0x20000, A=0x30000, B=0x40000, C=0x50000, D=0x60000, h0=None, dy=0x70000,
+                dhf=None, dx=0x80000, ddt=0x90000, dA=0xa0000, dB=0xb0000, dC=0xc0000, dD=0xd0000, dh0=None,
+                ws=0xe0000)
+
+
+def bwd_call(shape, ptrs, chunk=64, ws_bytes=1 << 34, dtype=B.SSD_BF16):
+    s = B.ShapeT(*shape)
+    p = {k: ctypes.c_void_p(v) if v else None for k, v in ptrs.items()}
+    return B.lib().ssd_bwd(ctypes.byref(s), dtype, p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], p["h0"], chunk,
+                           p["dy"], p["dhf"], p["dx"], p["ddt"], p["dA"], p["dB"], p["dC"], p["dD"], p["dh0"],
+                           p["ws"], ws_bytes, None)
+
+
+def test_bwd_workspace_bytes(lib):
+    out = ctypes.c_size_t(0)
+    shp = B.ShapeT(4, 8192, 80, 64, 1, 128)
+    assert lib.ssd_bwd_workspace_bytes(ctypes.byref(shp), B.SSD_BF16, 256, ctypes.byref(out)) == 0
+    # recomputed entering states and their gradients, [B,H,nc,P,N] fp32 each, dominate
+    assert out.value >= 2 * 4 * 80 * 32 * 64 * 128 * 4
+    assert lib.ssd_bwd_workspace_bytes(ctypes.byref(B.ShapeT(4, 0, 80, 64, 1, 128)), 1, 256, ctypes.byref(out)) == 0
+    assert out.value == 0
+    assert lib.ssd_bwd_workspace_bytes(ctypes.byref(shp), 1, 256, None) == 1
+    assert lib.ssd_bwd_workspace_bytes(ctypes.byref(B.ShapeT(1, 10, 4, 16, 3, 16)), 1, 64, ctypes.byref(out)) == 1
+
+
+def test_bwd_rejects_before_launch(lib):
+    shape = (2, 100, 4, 16, 2, 16)
+    for k in ("x", "dt", "A", "B", "C", "dy", "dx", "ddt", "dA", "dB", "dC"):
+        assert bwd_call(shape, {**BWD_GOOD, k: None}) == 1, k
+    for k in ("x", "dt", "A", "B", "C", "D", "dy", "dx", "ddt", "dA", "dB", "dC", "dD", "ws"):
+        assert bwd_call(shape, {**BWD_GOOD, k: BWD_GOOD[k] + 4}) == 3, k
+    assert bwd_call(shape, {**BWD_GOOD, "h0": 0xf0004}) == 3
+    assert bwd_call(shape, {**BWD_GOOD, "dhf": 0xf0008}) == 3
+    assert bwd_call(shape, {**BWD_GOOD, "dh0": 0xf000c}) == 3
+    assert bwd_call(shape, {**BWD_GOOD, "ws": None}) == 4
+    assert bwd_call(shape, BWD_GOOD, ws_bytes=16) == 4
+    assert bwd_call((2, 100, 4, 16, 3, 16), BWD_GOOD) == 1
+    assert bwd_call((2, 100, 4, 300, 1, 16), BWD_GOOD) == 2
+    assert bwd_call(shape, BWD_GOOD, chunk=0) == 1
+    assert bwd_call(shape, BWD_GOOD, chunk=257) == 2
+    assert bwd_call(shape, BWD_GOOD, dtype=3) == 1
 
 
 def test_verify_and_select_reject_before_launch(lib):
