@@ -398,7 +398,8 @@ def bwd_main(args, wl):
            "dB": torch.empty_like(g["B"]), "dC": torch.empty_like(g["C"]), "dD": torch.empty_like(g["D"]),
            "dh0": torch.empty_like(g["dhf"])}
     stream = torch.cuda.current_stream(dev)
-    launches = 11
+    plan = ssd.bwd_plan(wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.ngroups, wl.dstate, code, wl.chunk)
+    launches = plan["kernels"]
 
     def call(src):
         ssd.ssd_bwd(src["x"], src["dt"], src["A"], src["B"], src["C"], src["D"], h0, src["dy"], src["dhf"],
@@ -454,8 +455,13 @@ def bwd_main(args, wl):
     nbytes, flops = bwd_algorithmic(wl)
     hbm, tf, src = peaks()
     clk_mhz = clk.get("sm_mhz") or 1965.0
-    alu = alu_peak_tflops(clk.get("sm_max_mhz") or 1965.0)
     achieved = flops / (ms * 1e-3) / 1e12
+    if plan["path"] == "mma":  # every product on tensor cores (bf16 mma.sync)
+        bound, peak, peak_src = "tensor", tf, f"bf16 dense, {src} (MEASURED_PEAKS.json)"
+        what = "fp32-accumulated bf16 mma.sync products"
+    else:
+        bound, peak = "alu", alu_peak_tflops(clk.get("sm_max_mhz") or 1965.0)
+        peak_src, what = "148 SMs x 128 fp32 lanes x 2 FLOP x max SM clock", "fp32 FMA on CUDA cores"
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         v, n, threads, t = time_oracle(wl, d, args.cpu_seconds, backward=cot)
@@ -466,15 +472,16 @@ def bwd_main(args, wl):
         line = {
             "metric": BWD_METRIC, "value": tokens * ws / (ms_max * 1e-3), "unit": UNIT, "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": wl.name + " backward", "batch": wl.batch, "seqlen": wl.seqlen,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if plan["path"] == "mma" else "f32",
+            "data": "synthetic",
+            "config": {"workload": wl.name + " backward", "path": plan["path"], "batch": wl.batch, "seqlen": wl.seqlen,
                        "nheads": wl.nheads, "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups,
                        "chunk": wl.chunk, "io_dtype": wl.dtype,
                        "l2": "inputs larger than L2 (x, dy, dx 335.5 MB each per step vs 126 MB L2); no flush"},
-            "roofline": {"bound": "alu", "achieved": achieved, "peak": alu, "unit": "TFLOP/s",
-                         "frac": achieved / alu, "traffic": None,
-                         "kernel": "whole ssd_bwd call (%d launches, fp32 FMA on CUDA cores)" % launches,
-                         "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x max SM clock",
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "kernel": "whole ssd_bwd call (%d launches, %s)" % (launches, what),
+                         "peak_source": peak_src,
                          "alg_flops": flops, "alg_bytes": nbytes,
                          "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / hbm,
                          "tensor_roofline_ms": flops / (tf * 1e12) * 1e3,

@@ -70,6 +70,7 @@ typedef enum ssd_path_t {
     SSD_PATH_NONE = 0,    /* nothing to compute (batch == 0 or seqlen == 0) */
     SSD_PATH_SIMT = 1,    /* chunked, fp32 CUDA-core arithmetic, one kernel per step */
     SSD_PATH_TCGEN05 = 2, /* chunked, fused, bf16 tcgen05 tensor-core MMAs */
+    SSD_PATH_MMA = 3,     /* chunked, bf16 mma.sync tensor-core products (ssd_bwd) */
 } ssd_path_t;
 
 typedef struct ssd_plan_t {
@@ -299,6 +300,10 @@ ssd_status_t ssd_cp_correct(const ssd_shape_t *shape, ssd_dtype_t dtype, const v
  */
 ssd_status_t ssd_bwd_workspace_bytes(const ssd_shape_t *shape, ssd_dtype_t dtype, int64_t chunk,
                                      size_t *bytes);
+/* What ssd_bwd would launch: SSD_PATH_MMA (bf16 inputs with (headdim, dstate) in {(32, 64),
+ * (64, 64), (64, 128), (64, 256), (128, 128)}: every product on tensor cores, bf16 operands,
+ * fp32 accumulation), SSD_PATH_SIMT (everything else: fp32 CUDA cores) or SSD_PATH_NONE. */
+ssd_status_t ssd_bwd_plan(const ssd_shape_t *shape, ssd_dtype_t dtype, int64_t chunk, ssd_plan_t *plan);
 ssd_status_t ssd_bwd(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *x, const void *dt,
                      const float *A, const void *Bm, const void *Cm, const float *D, const float *h0,
                      int64_t chunk, const void *dy, const float *dh_final, void *dx, void *ddt,

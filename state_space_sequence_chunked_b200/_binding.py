@@ -34,7 +34,7 @@ class PlanT(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("kernels", ctypes.c_int32), ("workspace_bytes", ctypes.c_size_t)]
 
 
-PATHS = {0: "none", 1: "simt", 2: "tcgen05"}
+PATHS = {0: "none", 1: "simt", 2: "tcgen05", 3: "mma"}
 
 _lib = None
 _vp, _i64, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
@@ -51,6 +51,7 @@ _SIGS = {
     "ssd_cp_combine": ([ctypes.POINTER(ShapeT), _i64, _i64] + [_vp] * 5, ctypes.c_int),
     "ssd_cp_correct": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 8, ctypes.c_int),
     "ssd_bwd_workspace_bytes": ([ctypes.POINTER(ShapeT), ctypes.c_int, _i64, ctypes.POINTER(_sz)], ctypes.c_int),
+    "ssd_bwd_plan": ([ctypes.POINTER(ShapeT), ctypes.c_int, _i64, ctypes.POINTER(PlanT)], ctypes.c_int),
     "ssd_bwd": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 7 + [_i64] + [_vp] * 9 + [_vp, _sz, _vp],
                 ctypes.c_int),
 }
@@ -265,6 +266,15 @@ def bwd_workspace_bytes(batch, seqlen, nheads, headdim, ngroups, dstate, dtype_c
     _check(lib().ssd_bwd_workspace_bytes(ctypes.byref(shape), dtype_code, chunk, ctypes.byref(out)),
            "ssd_bwd_workspace_bytes")
     return out.value
+
+
+def bwd_plan(batch, seqlen, nheads, headdim, ngroups, dstate, dtype_code, chunk) -> dict:
+    """{'path': 'simt'|'mma'|'none', 'kernels': launches per call, 'workspace_bytes': int}."""
+    shape = ShapeT(batch, seqlen, nheads, headdim, ngroups, dstate)
+    out = PlanT()
+    _check(lib().ssd_bwd_plan(ctypes.byref(shape), dtype_code, chunk, ctypes.byref(out)), "ssd_bwd_plan")
+    return {"path": PATHS.get(out.path, str(out.path)), "kernels": out.kernels,
+            "workspace_bytes": out.workspace_bytes}
 
 
 def ssd_bwd(x, dt, A, B, C, D, h0, dy, dh_final=None, *, chunk: int, want_dD: bool = True,

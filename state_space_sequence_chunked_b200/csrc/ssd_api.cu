@@ -284,6 +284,24 @@ SSD_API ssd_status_t ssd_bwd_workspace_bytes(const ssd_shape_t *shape, ssd_dtype
     return SSD_OK;
 }
 
+SSD_API ssd_status_t ssd_bwd_plan(const ssd_shape_t *shape, ssd_dtype_t dtype, int64_t chunk, ssd_plan_t *plan) {
+    if (!plan) return SSD_ERR_INVALID_ARG;
+    FwdProblem p;
+    const ssd_status_t st = make_fwd(shape, dtype, chunk, &p);
+    if (st != SSD_OK) return st;
+    if (!simt_bwd_supported(p)) return SSD_ERR_UNSUPPORTED;
+    ssd_plan_t out{};
+    if (p.B == 0 || p.L == 0) {
+        out.path = SSD_PATH_NONE;
+    } else {
+        out.path = mma_bwd_supported(p) ? SSD_PATH_MMA : SSD_PATH_SIMT;
+        out.kernels = 11;
+        out.workspace_bytes = simt_bwd_workspace_bytes(p);
+    }
+    *plan = out;
+    return SSD_OK;
+}
+
 SSD_API ssd_status_t ssd_bwd(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *x, const void *dt,
                              const float *A, const void *Bm, const void *Cm, const float *D,
                              const float *h0, int64_t chunk, const void *dy, const float *dh_final,

@@ -32,6 +32,7 @@ constexpr int kMaxCol = 8;       // column blocks of 32: P, N <= 256
 
 struct BwdWs {
     float *acs, *dtw, *states, *dstates, *hfin, *dcs, *ddt_dir, *dB, *dC, *hterm, *dDpart, *dAbh, *dDbh;
+    float *kq, *rq, *uq, *tq, *ec;  // chunk-local pieces of the log-decay gradient (tensor-core path)
 };
 
 size_t n_chunk_rows(const FwdProblem &p) { return (size_t)(p.B * p.H * p.nc * p.Q); }
@@ -61,6 +62,11 @@ BwdWs carve(const FwdProblem &p, void *ws, size_t *total) {
     w.dDpart = take(BH * (size_t)p.nc * (size_t)n_row_tiles(p));
     w.dAbh = take(BH);
     w.dDbh = take(BH);
+    w.kq = take(n_chunk_rows(p));
+    w.rq = take(n_chunk_rows(p));
+    w.uq = take(n_chunk_rows(p));
+    w.tq = take(n_chunk_rows(p));
+    w.ec = take(BH * (size_t)p.nc);
     if (total) *total = off;
     return w;
 }
@@ -73,10 +79,13 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // Reverse state pass. grid (ceil(P*N/256), H, B). R[c] (in dstates) is replaced by Gend[c].
 // Also hterm[b,h] = <dh_final, h_final>, the last token's extra log-decay gradient.
+// With ec != NULL (the tensor-core path) also ec[b,h,c] += <Gend[c], S_in[c]> (s_in = the
+// entering states).
 __global__ void __launch_bounds__(kThreads)
     k_dstate_pass(const float *__restrict__ acs, const float *__restrict__ dh_final,
-                  const float *__restrict__ hfin, int H, int PN, int Q, int nc, float *__restrict__ dstates,
-                  float *__restrict__ dh0, float *__restrict__ hterm) {
+                  const float *__restrict__ hfin, const float *__restrict__ s_in, int H, int PN, int Q, int nc,
+                  float *__restrict__ dstates, float *__restrict__ dh0, float *__restrict__ hterm,
+                  float *__restrict__ ec) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     const int h = blockIdx.y, b = blockIdx.z;
     const int64_t bh = (int64_t)b * H + h;
@@ -86,14 +95,30 @@ __global__ void __launch_bounds__(kThreads)
         const float part = warp_sum(valid ? run * hfin[bh * PN + e] : 0.f);
         if ((threadIdx.x & 31) == 0) atomicAdd(hterm + bh, part);
     }
-    if (!valid) return;
-    for (int c = nc - 1; c >= 0; --c) {
-        const int64_t idx = (bh * nc + c) * PN + e;
-        const float r = dstates[idx];
-        dstates[idx] = run;
-        run = fmaf(expf(acs[(bh * nc + c) * Q + Q - 1]), run, r);
+    // serial in c; the loads of 8 chunks are issued before the chain
+    for (int c1 = nc - 1; c1 >= 0; c1 -= 8) {
+        float r[8], dec[8], si[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int c = c1 - i;
+            r[i] = (valid && c >= 0) ? dstates[(bh * nc + c) * PN + e] : 0.f;
+            si[i] = (ec && valid && c >= 0) ? s_in[(bh * nc + c) * PN + e] : 0.f;
+            dec[i] = c >= 0 ? acs[(bh * nc + c) * Q + Q - 1] : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int c = c1 - i;
+            if (c >= 0) {
+                if (valid) dstates[(bh * nc + c) * PN + e] = run;
+                if (ec) {
+                    const float part = warp_sum(run * si[i]);
+                    if ((threadIdx.x & 31) == 0) atomicAdd(ec + bh * nc + c, part);
+                }
+                run = fmaf(expf(dec[i]), run, r[i]);
+            }
+        }
     }
-    if (dh0) dh0[bh * PN + e] = run;
+    if (valid && dh0) dh0[bh * PN + e] = run;
 }
 
 // Tokens as sources. grid (nc * nrt, H, B); a tile of 32 tokens s of one chunk.
@@ -499,6 +524,89 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// Tensor-core path: the log-decay gradient of token t from chunk-local pieces only,
+//   G_t = <Gbar_t, exp(a_t) S_{t-1}>
+//       = sum_{u<t} (K_u - R_u)            pairs s < t <= l of the chunk (K: row sums over l > s,
+//                                          R: column sums over s < l, of the same fp32 products)
+//       + sum_{l>=t} T_l                   T_l = exp(A_cs[l]) dy_l^T S_in C_l
+//       + sum_{s<t} U_s                    U_s = exp(A_cs[Q-1]-A_cs[s]) dt_s x_s^T Gend B_s
+//       + exp(A_cs[Q-1]) <Gend, S_in>
+// (the adjoint and the state of the recurrence written in the chunk's terms), then
+// ddt_t = A_h G_t + ddt_t(direct) and dA_h += dt_t G_t. grid (H, B); a chunk at a time,
+// thread l = token l of the chunk (Q <= 256).
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+    k_bwd_dt_local(const float *__restrict__ kq, const float *__restrict__ rq, const float *__restrict__ uq,
+                   const float *__restrict__ tq, const float *__restrict__ ec, const float *__restrict__ acs,
+                   const float *__restrict__ ddt_dir, const float *__restrict__ dtw, const float *__restrict__ dDpart,
+                   const float *__restrict__ A, int64_t L, int H, int Q, int nc, int nrt, T *__restrict__ ddt,
+                   float *__restrict__ dAbh, float *__restrict__ dDbh) {
+    __shared__ float wa[kThreads / 32], wb[kThreads / 32];
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int64_t bh = (int64_t)b * H + h;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const float Ah = A[h];
+    float da = 0.f;
+    for (int c = 0; c < nc; ++c) {
+        const int64_t t0 = (int64_t)c * Q;
+        const int q = (int)min((int64_t)Q, L - t0);
+        const int64_t lb = (bh * nc + c) * Q;
+        const bool ok = tid < q;
+        // prefix (exclusive) of K - R + U; suffix (inclusive) of T = total - exclusive prefix
+        float pv = ok ? kq[lb + tid] - rq[lb + tid] + uq[lb + tid] : 0.f;
+        float tv = ok ? tq[lb + tid] : 0.f;
+        float ip = pv, it = tv;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float a = __shfl_up_sync(0xffffffffu, ip, o), bb = __shfl_up_sync(0xffffffffu, it, o);
+            if (lane >= o) {
+                ip += a;
+                it += bb;
+            }
+        }
+        __syncthreads();
+        if (lane == 31) {
+            wa[warp] = ip;
+            wb[warp] = it;
+        }
+        __syncthreads();
+        float pre_p = 0.f, pre_t = 0.f, tot_t = 0.f;
+        for (int w = 0; w < kThreads / 32; ++w) {
+            if (w < warp) {
+                pre_p += wa[w];
+                pre_t += wb[w];
+            }
+            tot_t += wb[w];
+        }
+        const float excl_p = pre_p + ip - pv, excl_t = pre_t + it - tv;
+        const float G = excl_p + (tot_t - excl_t) + __expf(acs[lb + Q - 1]) * ec[bh * nc + c];
+        if (ok) {
+            const float dtv = dtw[lb + tid];
+            store_as(ddt + ((int64_t)b * L + t0 + tid) * H + h, fmaf(Ah, G, ddt_dir[lb + tid]));
+            da = fmaf(dtv, G, da);
+        }
+    }
+    float dd = 0.f;
+    for (int i = tid; i < nc * nrt; i += kThreads) dd += dDpart[bh * nc * nrt + i];
+    da = warp_sum(da);
+    dd = warp_sum(dd);
+    __syncthreads();
+    if (lane == 0) {
+        wa[warp] = da;
+        wb[warp] = dd;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float s1 = 0.f, s2 = 0.f;
+        for (int w = 0; w < kThreads / 32; ++w) {
+            s1 += wa[w];
+            s2 += wb[w];
+        }
+        dAbh[bh] = s1;
+        dDbh[bh] = s2;
+    }
+}
+
 // dA[h] = sum_b, dD[h] = sum_b (fixed order); dB/dC from the fp32 sums to the output dtype.
 __global__ void k_bwd_reduce_heads(const float *__restrict__ dAbh, const float *__restrict__ dDbh, int64_t B, int H,
                                    float *__restrict__ dA, float *__restrict__ dD) {
@@ -541,17 +649,36 @@ cudaError_t run(const FwdProblem &p, const BwdGrads &gr, void *ws, cudaStream_t 
     if ((e = cudaMemsetAsync(w.dB, 0, BLGN * sizeof(float), s))) return e;
     if ((e = cudaMemsetAsync(w.dC, 0, BLGN * sizeof(float), s))) return e;
     if ((e = cudaMemsetAsync(w.hterm, 0, BH * sizeof(float), s))) return e;
+    // bf16 inputs of a compiled (P, N) run every product on tensor cores (ssd_bwd_mma.cu)
+    const bool tc = mma_bwd_supported(p);
+    if (tc) {
+        if ((e = cudaMemsetAsync(w.rq, 0, n_chunk_rows(p) * sizeof(float), s))) return e;
+        if ((e = cudaMemsetAsync(w.ec, 0, BH * (size_t)nc * sizeof(float), s))) return e;
+    }
+    const int nrt_used = tc ? mma_row_tiles(p) : nrt;
     // recompute: A_cs, dt per chunk, S_in per chunk, h_final
-    if ((e = simt_states(p, w.acs, w.dtw, w.states, w.hfin, s))) return e;
-    // R[c], then the reverse state pass
-    if ((e = simt_adjoint_chunk_sums(p, gr.dy, w.acs, w.dstates, s))) return e;
+    if (tc) {
+        if ((e = simt_cumsum(p, w.acs, w.dtw, s))) return e;
+        if ((e = mma_chunk_sums(p, false, p.x, p.Bm, w.acs, w.dtw, w.states, s))) return e;
+        if ((e = simt_state_pass(p, w.acs, w.states, w.hfin, s))) return e;
+        if ((e = mma_chunk_sums(p, true, gr.dy, p.Cm, w.acs, w.dtw, w.dstates, s))) return e;
+    } else {
+        if ((e = simt_states(p, w.acs, w.dtw, w.states, w.hfin, s))) return e;
+        if ((e = simt_adjoint_chunk_sums(p, gr.dy, w.acs, w.dstates, s))) return e;
+    }
+    // R[c] (in dstates), then the reverse state pass
     {
         dim3 grid((P * N + kThreads - 1) / kThreads, H, (unsigned)p.B);
-        k_dstate_pass<<<grid, kThreads, 0, s>>>(w.acs, gr.dh_final, w.hfin, H, P * N, Q, nc, w.dstates, gr.dh0,
-                                                w.hterm);
+        k_dstate_pass<<<grid, kThreads, 0, s>>>(w.acs, gr.dh_final, w.hfin, w.states, H, P * N, Q, nc, w.dstates,
+                                                gr.dh0, w.hterm, tc ? w.ec : nullptr);
         if ((e = cudaGetLastError())) return e;
     }
-    {
+    if (tc) {
+        if ((e = mma_bwd_src(p, gr.dy, w.acs, w.dtw, w.dstates, gr.dx, w.dB, w.kq, w.rq, w.uq, w.ddt_dir, w.dDpart,
+                             s)))
+            return e;
+        if ((e = mma_bwd_dst(p, gr.dy, w.acs, w.dtw, w.states, w.dC, w.tq, s))) return e;
+    } else {
         const size_t smem = src_smem(p);
         if ((e = cudaFuncSetAttribute(k_bwd_src<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
             return e;
@@ -560,20 +687,23 @@ cudaError_t run(const FwdProblem &p, const BwdGrads &gr, void *ws, cudaStream_t 
                                                   nc, nrt, static_cast<T *>(gr.dx), w.dB, w.dcs, w.ddt_dir,
                                                   w.dDpart);
         if ((e = cudaGetLastError())) return e;
-    }
-    {
-        const size_t smem = dst_smem(p);
-        if ((e = cudaFuncSetAttribute(k_bwd_dst<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+        const size_t smem2 = dst_smem(p);
+        if ((e = cudaFuncSetAttribute(k_bwd_dst<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2)))
             return e;
-        dim3 grid(nc * nrt, H, (unsigned)p.B);
-        k_bwd_dst<T><<<grid, kThreads, smem, s>>>(x, Bm, Cm, dy, w.acs, w.dtw, w.states, p.L, H, P, G, N, Q, nc,
+        k_bwd_dst<T><<<grid, kThreads, smem2, s>>>(x, Bm, Cm, dy, w.acs, w.dtw, w.states, p.L, H, P, G, N, Q, nc,
                                                   nrt, w.dC, w.dcs);
         if ((e = cudaGetLastError())) return e;
     }
     {
         dim3 grid(H, (unsigned)p.B);
-        k_bwd_dt<T><<<grid, kThreads, 0, s>>>(w.dcs, w.ddt_dir, w.dtw, gr.dh_final ? w.hterm : nullptr, w.dDpart,
-                                              p.A, p.L, H, Q, nc, nrt, static_cast<T *>(gr.ddt), w.dAbh, w.dDbh);
+        if (tc)
+            k_bwd_dt_local<T><<<grid, kThreads, 0, s>>>(w.kq, w.rq, w.uq, w.tq, w.ec, w.acs, w.ddt_dir, w.dtw,
+                                                        w.dDpart, p.A, p.L, H, Q, nc, nrt_used,
+                                                        static_cast<T *>(gr.ddt), w.dAbh, w.dDbh);
+        else
+            k_bwd_dt<T><<<grid, kThreads, 0, s>>>(w.dcs, w.ddt_dir, w.dtw, gr.dh_final ? w.hterm : nullptr,
+                                                  w.dDpart, p.A, p.L, H, Q, nc, nrt_used, static_cast<T *>(gr.ddt),
+                                                  w.dAbh, w.dDbh);
         if ((e = cudaGetLastError())) return e;
     }
     k_bwd_reduce_heads<<<(H + 127) / 128, 128, 0, s>>>(w.dAbh, w.dDbh, p.B, H, gr.dA, gr.dD);

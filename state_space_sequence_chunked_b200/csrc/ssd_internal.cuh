@@ -52,6 +52,9 @@ cudaError_t simt_fwd(const FwdProblem &p, void *ws, cudaStream_t s);
 // steps 0, 2, 3 alone: A_cs [B,H,nc,Q], dt [B,H,nc,Q], entering states [B,H,nc,P,N], h_final
 cudaError_t simt_states(const FwdProblem &p, float *acs, float *dtw, float *states, float *h_final,
                         cudaStream_t s);
+// the two halves of simt_states around step 2: step 0, and step 3 (in place on `states`)
+cudaError_t simt_cumsum(const FwdProblem &p, float *acs, float *dtw, cudaStream_t s);
+cudaError_t simt_state_pass(const FwdProblem &p, const float *acs, float *states, float *h_final, cudaStream_t s);
 // out[b,h,c] = sum_{l in c} exp(A_cs[l]) dy_l C_l^T   (dy [B,L,H,P] in the input dtype)
 cudaError_t simt_adjoint_chunk_sums(const FwdProblem &p, const void *dy, const float *acs, float *out,
                                     cudaStream_t s);
@@ -60,6 +63,19 @@ cudaError_t simt_adjoint_chunk_sums(const FwdProblem &p, const void *dy, const f
 bool simt_bwd_supported(const FwdProblem &p);
 size_t simt_bwd_workspace_bytes(const FwdProblem &p);
 cudaError_t simt_bwd(const FwdProblem &p, const BwdGrads &g, void *ws, cudaStream_t s);
+// bf16 tensor-core (mma.sync) kernels of the backward, for the (P, N) pairs mma_bwd_supported
+// accepts. Chunk sums: forward (x, B, exp(A_cs[Q-1] - A_cs[l]) dt_l) or adjoint (dy, C, exp(A_cs[l])).
+bool mma_bwd_supported(const FwdProblem &p);
+cudaError_t mma_chunk_sums(const FwdProblem &p, bool adjoint, const void *u, const void *v, const float *acs,
+                           const float *dtw, float *out, cudaStream_t s);
+// Sources: dx, dB (atomics), x.u, and per token K_s, U_s and (atomics) R_l; targets: dC
+// (atomics) and T_l; the chunk-local pieces of the log-decay gradient (see ssd_bwd.cu).
+cudaError_t mma_bwd_src(const FwdProblem &p, const void *dy, const float *acs, const float *dtw, const float *gend,
+                        void *dx, float *dB_acc, float *kq, float *rq, float *uq, float *ddt_dir, float *dDpart,
+                        cudaStream_t s);
+cudaError_t mma_bwd_dst(const FwdProblem &p, const void *dy, const float *acs, const float *dtw, const float *s_in,
+                        float *dC_acc, float *tq, cudaStream_t s);
+int mma_row_tiles(const FwdProblem &p);
 
 // ---- fused chunked path on tcgen05 tensor cores (bf16, P = 64, N in {128, 256}) ----
 bool tc_supported(const FwdProblem &p);

@@ -154,11 +154,23 @@ __global__ void __launch_bounds__(kThreads)
     if (e >= PN) return;
     const int64_t bh = (int64_t)b * H + h;
     float run = h0 ? h0[bh * PN + e] : 0.f;
-    for (int c = 0; c < nc; ++c) {
-        const int64_t idx = (bh * nc + c) * PN + e;
-        const float sc = states[idx];
-        states[idx] = run;
-        run = fmaf(expf(acs[(bh * nc + c) * Q + Q - 1]), run, sc);
+    // the chain is serial in c; the loads of 8 chunks are issued before it
+    for (int c0 = 0; c0 < nc; c0 += 8) {
+        float sc[8], dec[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int c = c0 + i;
+            sc[i] = c < nc ? states[(bh * nc + c) * PN + e] : 0.f;
+            dec[i] = c < nc ? acs[(bh * nc + c) * Q + Q - 1] : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int c = c0 + i;
+            if (c < nc) {
+                states[(bh * nc + c) * PN + e] = run;
+                run = fmaf(expf(dec[i]), run, sc[i]);
+            }
+        }
     }
     if (h_final) h_final[bh * PN + e] = run;
 }
@@ -353,6 +365,32 @@ size_t simt_fwd_workspace_bytes(const FwdProblem &p) {
 
 cudaError_t simt_fwd(const FwdProblem &p, void *ws, cudaStream_t s) {
     return p.dtype == SSD_F32 ? run<float>(p, ws, s) : run<__nv_bfloat16>(p, ws, s);
+}
+
+cudaError_t simt_cumsum(const FwdProblem &p, float *acs, float *dtw, cudaStream_t s) {
+    const int H = (int)p.H, Q = (int)p.Q, nc = (int)p.nc;
+    const size_t smem = (size_t)Q * 33 * sizeof(float);
+    dim3 grid(nc, (H + 31) / 32, (unsigned)p.B);
+    cudaError_t e;
+    if (p.dtype == SSD_F32) {
+        if ((e = cudaFuncSetAttribute(k_cumsum<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+            return e;
+        k_cumsum<float><<<grid, kThreads, smem, s>>>(static_cast<const float *>(p.dt), p.A, p.L, H, Q, nc, acs, dtw);
+    } else {
+        if ((e = cudaFuncSetAttribute(k_cumsum<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)))
+            return e;
+        k_cumsum<__nv_bfloat16><<<grid, kThreads, smem, s>>>(static_cast<const __nv_bfloat16 *>(p.dt), p.A, p.L, H,
+                                                             Q, nc, acs, dtw);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t simt_state_pass(const FwdProblem &p, const float *acs, float *states, float *h_final, cudaStream_t s) {
+    const int P = (int)p.P, N = (int)p.N;
+    dim3 grid((P * N + kThreads - 1) / kThreads, (unsigned)p.H, (unsigned)p.B);
+    k_state_pass<<<grid, kThreads, 0, s>>>(acs, p.h0, (int)p.H, P * N, (int)p.Q, (int)p.nc, states, h_final);
+    return cudaGetLastError();
 }
 
 cudaError_t simt_states(const FwdProblem &p, float *acs, float *dtw, float *states, float *h_final,

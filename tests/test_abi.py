@@ -137,6 +137,18 @@ def test_bwd_workspace_bytes(lib):
     assert lib.ssd_bwd_workspace_bytes(ctypes.byref(B.ShapeT(1, 10, 4, 16, 3, 16)), 1, 64, ctypes.byref(out)) == 1
 
 
+def test_bwd_plan_selects_path(lib):
+    def plan(shape, dtype):
+        out = B.PlanT()
+        st = lib.ssd_bwd_plan(ctypes.byref(B.ShapeT(*shape)), dtype, 256, ctypes.byref(out))
+        return st, out.path, out.kernels
+    assert plan((4, 8192, 80, 64, 1, 128), B.SSD_BF16) == (0, 3, 11)   # tensor cores
+    assert plan((4, 8192, 80, 64, 1, 128), B.SSD_F32) == (0, 1, 11)    # fp32 inputs: CUDA cores
+    assert plan((1, 90, 2, 200, 1, 40), B.SSD_BF16) == (0, 1, 11)     # no compiled (P, N) instance
+    assert plan((1, 0, 2, 64, 1, 128), B.SSD_BF16)[:2] == (0, 0)
+    assert lib.ssd_bwd_plan(ctypes.byref(B.ShapeT(1, 1, 1, 1, 1, 1)), 0, 1, None) == 1
+
+
 def test_bwd_rejects_before_launch(lib):
     shape = (2, 100, 4, 16, 2, 16)
     for k in ("x", "dt", "A", "B", "C", "dy", "dx", "ddt", "dA", "dB", "dC"):
