@@ -300,9 +300,9 @@ ssd_status_t ssd_cp_correct(const ssd_shape_t *shape, ssd_dtype_t dtype, const v
  */
 ssd_status_t ssd_bwd_workspace_bytes(const ssd_shape_t *shape, ssd_dtype_t dtype, int64_t chunk,
                                      size_t *bytes);
-/* What ssd_bwd would launch: SSD_PATH_MMA (bf16 inputs with (headdim, dstate) in {(32, 64),
- * (64, 64), (64, 128), (64, 256), (128, 128)}: every product on tensor cores, bf16 operands,
- * fp32 accumulation), SSD_PATH_SIMT (everything else: fp32 CUDA cores) or SSD_PATH_NONE. */
+/* What ssd_bwd would launch: SSD_PATH_MMA (bf16 inputs with (headdim, dstate) in {(64, 64),
+ * (64, 128), (64, 256), (128, 128)}: every product on tensor cores, bf16 operands, fp32
+ * accumulation), SSD_PATH_SIMT (everything else: fp32 CUDA cores) or SSD_PATH_NONE. */
 ssd_status_t ssd_bwd_plan(const ssd_shape_t *shape, ssd_dtype_t dtype, int64_t chunk, ssd_plan_t *plan);
 ssd_status_t ssd_bwd(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *x, const void *dt,
                      const float *A, const void *Bm, const void *Cm, const float *D, const float *h0,

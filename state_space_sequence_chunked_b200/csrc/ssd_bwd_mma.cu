@@ -19,7 +19,8 @@ namespace ssd {
 namespace {
 
 constexpr int kT = 64;        // tokens per tile
-constexpr int kThr = 256;     // 8 warps
+constexpr int kThr = 256;     // 8 warps (chunk sums)
+constexpr int kThr2 = 512;    // 16 warps (source and target kernels)
 
 typedef __nv_bfloat16 bf16;
 
@@ -64,9 +65,10 @@ __device__ __forceinline__ uint32_t b_kn(uint32_t base, int ld, int n0, int k0, 
 // rows [r0, r0 + 64) of a [rows][W] bf16 matrix (row stride `gstride` elements in global) into
 // shared [64][W + 8]; rows >= nrows are zero. W % 8 == 0, 16-byte aligned rows.
 template <int W>
-__device__ __forceinline__ void load_rows(bf16 *dst, const bf16 *src, int64_t gstride, int nrows, int tid) {
+__device__ __forceinline__ void load_rows(bf16 *dst, const bf16 *src, int64_t gstride, int nrows, int tid,
+                                          int nthr) {
     constexpr int V = W / 8;
-    for (int i = tid; i < kT * V; i += kThr) {
+    for (int i = tid; i < kT * V; i += nthr) {
         const int r = i / V, c = i % V;
         bf16 *d = dst + r * (W + 8) + 8 * c;
         if (r < nrows) {
@@ -84,9 +86,9 @@ __device__ __forceinline__ void async_wait() {
 
 // fp32 [P][N] (global) to bf16 [P][N + 8] (shared)
 template <int P, int N>
-__device__ __forceinline__ void load_state_bf16(bf16 *dst, const float *src, int tid) {
+__device__ __forceinline__ void load_state_bf16(bf16 *dst, const float *src, int tid, int nthr) {
     constexpr int V = N / 4;
-    for (int i = tid; i < P * V; i += kThr) {
+    for (int i = tid; i < P * V; i += nthr) {
         const int r = i / V, c = i % V;
         const float4 v = reinterpret_cast<const float4 *>(src)[i];
         __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
@@ -130,7 +132,7 @@ __global__ void __launch_bounds__(kThr)
     for (int l0 = 0; l0 < q; l0 += kT) {
         const int nl = min(kT, q - l0);
         __syncthreads();
-        load_rows<N>(vs, v + (((int64_t)b * L + t0 + l0) * G + g) * N, (int64_t)G * N, nl, tid);
+        load_rows<N>(vs, v + (((int64_t)b * L + t0 + l0) * G + g) * N, (int64_t)G * N, nl, tid, kThr);
         // u rows scaled by their weight, rounded to bf16
         constexpr int V = P / 8;
         for (int i = tid; i < kT * V; i += kThr) {
@@ -176,9 +178,11 @@ __global__ void __launch_bounds__(kThr)
 }
 
 // ---- tokens as sources --------------------------------------------------------------
-// grid (nc * nrt, H, B); tile of 64 tokens s. Warp w: rows 16 (w & 3) .., column half w >> 2.
+// grid (nc * nrt, H, B); a tile of 64 tokens s per CTA, 16 warps. Warp w: rows 16 (w & 3) ..,
+// column quarter w >> 2 of u and v, and columns 16 (w >> 2) .. of each 64 x 64 W tile. The next
+// target tile's C and dy rows load (cp.async, double buffer) while this one is multiplied.
 template <int P, int N>
-__global__ void __launch_bounds__(kThr, 1)
+__global__ void __launch_bounds__(kThr2, 1)
     k_bwd_src_mma(const bf16 *__restrict__ x, const bf16 *__restrict__ Bm, const bf16 *__restrict__ Cm,
                   const bf16 *__restrict__ dy, const float *__restrict__ acs, const float *__restrict__ dtw,
                   const float *__restrict__ gend, const float *__restrict__ D, int64_t L, int H, int G, int Q, int nc,
@@ -186,19 +190,20 @@ __global__ void __launch_bounds__(kThr, 1)
                   float *__restrict__ rq, float *__restrict__ uq, float *__restrict__ ddt_dir,
                   float *__restrict__ dDpart) {
     constexpr int LN = N + 8, LP = P + 8, LW = kT + 8;
-    constexpr int TU = P / 16, TV = N / 16;  // n8 tiles per warp (half the columns)
+    constexpr int TU = P / 32, TV = N / 32;  // n8 tiles per warp (a quarter of the columns)
+    static_assert(TU % 2 == 0 && TV % 2 == 0, "column quarters are whole n16 pairs");
     extern __shared__ __align__(16) unsigned char smem[];
-    bf16 *bs = reinterpret_cast<bf16 *>(smem);  // [64][LN]  B_s
-    bf16 *xs = bs + kT * LN;                     // [64][LP]  x_s
-    bf16 *cl = xs + kT * LP;                     // [64][LN]  C_l
-    bf16 *dl = cl + kT * LN;                     // [64][LP]  dy_l
-    bf16 *w1 = dl + kT * LP;                     // [64][LW]  W1^T [s][l]
-    bf16 *w2 = w1 + kT * LW;                     // [64][LW]  W2^T [s][l]
-    bf16 *ge = w2 + kT * LW;                     // [P][LN]   Gend
+    bf16 *bs = reinterpret_cast<bf16 *>(smem);  // [64][LN]     B_s
+    bf16 *xs = bs + kT * LN;                     // [64][LP]     x_s
+    bf16 *cl = xs + kT * LP;                     // [2][64][LN]  C_l (double buffer)
+    bf16 *dl = cl + 2 * kT * LN;                 // [2][64][LP]  dy_l
+    bf16 *w1 = dl + 2 * kT * LP;                 // [64][LW]     W1^T [s][l]
+    bf16 *w2 = w1 + kT * LW;                     // [64][LW]     W2^T [s][l]
+    bf16 *ge = w2 + kT * LW;                     // [P][LN]      Gend
     float *as = reinterpret_cast<float *>(ge + P * LN);  // [64]
-    float *al = as + kT;                                 // [64]
-    float *ds = al + kT;                                 // [64] dt_s
-    float *red = ds + kT;                                // [2][64] x 3 + [8]
+    float *al = as + kT;                                 // [2][64]
+    float *ds = al + 2 * kT;                             // [64] dt_s
+    float *red = ds + kT;                                // [3][4][64] + [16]
 
     const int c = blockIdx.x / nrt, rt = blockIdx.x % nrt, r0 = rt * kT;
     const int h = blockIdx.y, b = blockIdx.z, g = h / (H / G);
@@ -211,20 +216,23 @@ __global__ void __launch_bounds__(kThr, 1)
         return;
     }
     const int nr = min(kT, q - r0);
-    load_rows<N>(bs, Bm + (((int64_t)b * L + t0 + r0) * G + g) * N, (int64_t)G * N, nr, tid);
-    load_rows<P>(xs, x + (((int64_t)b * L + t0 + r0) * H + h) * P, (int64_t)H * P, nr, tid);
-    load_state_bf16<P, N>(ge, gend + (bh * nc + c) * (int64_t)P * N, tid);
-    for (int i = tid; i < kT; i += kThr) {
+    load_rows<N>(bs, Bm + (((int64_t)b * L + t0 + r0) * G + g) * N, (int64_t)G * N, nr, tid, kThr2);
+    load_rows<P>(xs, x + (((int64_t)b * L + t0 + r0) * H + h) * P, (int64_t)H * P, nr, tid, kThr2);
+    load_rows<N>(cl, Cm + (((int64_t)b * L + t0 + r0) * G + g) * N, (int64_t)G * N, nr, tid, kThr2);
+    load_rows<P>(dl, dy + (((int64_t)b * L + t0 + r0) * H + h) * P, (int64_t)H * P, nr, tid, kThr2);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    load_state_bf16<P, N>(ge, gend + (bh * nc + c) * (int64_t)P * N, tid, kThr2);
+    for (int i = tid; i < kT; i += kThr2) {
         as[i] = acs[lb + min(r0 + i, Q - 1)];
+        al[i] = as[i];
         ds[i] = i < nr ? dtw[lb + r0 + i] : 0.f;
     }
-    async_wait();
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();
 
-    const int rb = warp & 3, ch = warp >> 2;
-    const int pu0 = ch * (P / 2), nv0 = ch * (N / 2);
-    const uint32_t bsb = su32(bs), xsb = su32(xs), clb = su32(cl), dlb = su32(dl), w1b = su32(w1), w2b = su32(w2),
-                   geb = su32(ge);
+    const int rb = warp & 3, cq = warp >> 2;
+    const int pu0 = cq * (P / 4), nv0 = cq * (N / 4);
+    const uint32_t bsb = su32(bs), xsb = su32(xs), w1b = su32(w1), w2b = su32(w2), geb = su32(ge);
     float au[TU][4], av[TV][4];
 #pragma unroll
     for (int j = 0; j < TU; ++j)
@@ -289,60 +297,63 @@ __global__ void __launch_bounds__(kThr, 1)
     float kpart[2] = {0.f, 0.f};  // K_s over the target tiles, rows rlo, rhi
 
     // within the chunk: target tiles l >= s
-    const int wr = warp & 3, wc = (warp >> 2) * 32;  // W tile split: rows 16 wr, columns wc .. wc + 31
-    for (int l0 = r0; l0 < q; l0 += kT) {
-        const int nl = min(kT, q - l0);
+    const int wc = cq * 16;  // this warp's 16 columns l of a W tile (rows 16 rb ..)
+    int it = 0;
+    for (int l0 = r0; l0 < q; l0 += kT, ++it) {
+        const int cur = it & 1, nl = min(kT, q - l0);
+        bf16 *clc = cl + cur * kT * LN, *dlc = dl + cur * kT * LP;
+        const float *alc = al + cur * kT;
+        const int l1 = l0 + kT;
+        if (l1 < q) {  // prefetch the next target tile into the other buffer
+            const int n1 = min(kT, q - l1);
+            load_rows<N>(cl + (cur ^ 1) * kT * LN, Cm + (((int64_t)b * L + t0 + l1) * G + g) * N, (int64_t)G * N, n1,
+                         tid, kThr2);
+            load_rows<P>(dl + (cur ^ 1) * kT * LP, dy + (((int64_t)b * L + t0 + l1) * H + h) * P, (int64_t)H * P, n1,
+                         tid, kThr2);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            for (int i = tid; i < kT; i += kThr2) al[(cur ^ 1) * kT + i] = acs[lb + min(l1 + i, Q - 1)];
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
         __syncthreads();
-        load_rows<N>(cl, Cm + (((int64_t)b * L + t0 + l0) * G + g) * N, (int64_t)G * N, nl, tid);
-        load_rows<P>(dl, dy + (((int64_t)b * L + t0 + l0) * H + h) * P, (int64_t)H * P, nl, tid);
-        for (int i = tid; i < kT; i += kThr) al[i] = acs[lb + min(l0 + i, Q - 1)];
-        async_wait();
-        __syncthreads();
-        float f1[4][4], f2[4][4];
+        const uint32_t clb = su32(clc), dlb = su32(dlc);
+        float f1[2][4], f2[2][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) f1[j][e] = f2[j][e] = 0.f;
-#pragma unroll 2
+#pragma unroll 4
         for (int k0 = 0; k0 < N; k0 += 16) {
-            uint32_t a[4];
-            ldsm4(a_mk(bsb, LN, 16 * wr, k0, lane), a);
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                uint32_t bb[4];
-                ldsm4(b_nk(clb, LN, wc + 16 * jj, k0, lane), bb);
-                mma(f1[2 * jj], a, bb[0], bb[1]);
-                mma(f1[2 * jj + 1], a, bb[2], bb[3]);
-            }
+            uint32_t a[4], bb[4];
+            ldsm4(a_mk(bsb, LN, 16 * rb, k0, lane), a);
+            ldsm4(b_nk(clb, LN, wc, k0, lane), bb);
+            mma(f1[0], a, bb[0], bb[1]);
+            mma(f1[1], a, bb[2], bb[3]);
         }
-#pragma unroll 2
+#pragma unroll 4
         for (int k0 = 0; k0 < P; k0 += 16) {
-            uint32_t a[4];
-            ldsm4(a_mk(xsb, LP, 16 * wr, k0, lane), a);
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                uint32_t bb[4];
-                ldsm4(b_nk(dlb, LP, wc + 16 * jj, k0, lane), bb);
-                mma(f2[2 * jj], a, bb[0], bb[1]);
-                mma(f2[2 * jj + 1], a, bb[2], bb[3]);
-            }
+            uint32_t a[4], bb[4];
+            ldsm4(a_mk(xsb, LP, 16 * rb, k0, lane), a);
+            ldsm4(b_nk(dlb, LP, wc, k0, lane), bb);
+            mma(f2[0], a, bb[0], bb[1]);
+            mma(f2[1], a, bb[2], bb[3]);
         }
         // mask l >= s (and the tile ends), decay exp(A_cs[l] - A_cs[s]), to bf16; and the fp32
         // pair products M (strictly l > s): row sums into K_s, column sums into R_l
         {
-            const int slo = 16 * wr + (lane >> 2);
-            float rcol[4][2];
+            float rcol[2][2];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 2; ++j) {
                 const int lc = wc + 8 * j + 2 * (lane & 3);
                 rcol[j][0] = rcol[j][1] = 0.f;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-                    const int s = slo + 8 * hf;
+                    const int s = rlo + 8 * hf;
                     float d0 = 0.f, d1 = 0.f;
                     if (s < nr) {
-                        if (lc < nl && l0 + lc >= r0 + s) d0 = __expf(al[lc] - as[s]);
-                        if (lc + 1 < nl && l0 + lc + 1 >= r0 + s) d1 = __expf(al[lc + 1] - as[s]);
+                        if (lc < nl && l0 + lc >= r0 + s) d0 = __expf(alc[lc] - as[s]);
+                        if (lc + 1 < nl && l0 + lc + 1 >= r0 + s) d1 = __expf(alc[lc + 1] - as[s]);
                     }
                     *reinterpret_cast<uint32_t *>(w1 + s * LW + lc) = pack2(f1[j][2 * hf] * d0, f1[j][2 * hf + 1] * d1);
                     *reinterpret_cast<uint32_t *>(w2 + s * LW + lc) = pack2(f2[j][2 * hf] * d0, f2[j][2 * hf + 1] * d1);
@@ -353,9 +364,8 @@ __global__ void __launch_bounds__(kThr, 1)
                     rcol[j][1] += m1;
                 }
             }
-            // column sums over the 8 row groups of the warp, then one atomic per column per warp
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
                 for (int e2 = 0; e2 < 2; ++e2) {
                     float v = rcol[j][e2];
@@ -388,6 +398,7 @@ __global__ void __launch_bounds__(kThr, 1)
                 mma(av[2 * jj + 1], a, bb[2], bb[3]);
             }
         }
+        __syncthreads();  // this tile's buffers and W are free for the next iteration
     }
 
     // epilogue
@@ -418,7 +429,7 @@ __global__ void __launch_bounds__(kThr, 1)
             atomicAdd(reinterpret_cast<float2 *>(dbrow + n), make_float2(dts * av[j][2 * hf], dts * av[j][2 * hf + 1]));
         }
     }
-    // row sums: the 4 lanes of a row, then the two column halves through shared memory
+    // row sums: the 4 lanes of a row, then the four column quarters through shared memory
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
@@ -430,49 +441,51 @@ __global__ void __launch_bounds__(kThr, 1)
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
-    float *rxu = red, *rk = red + 2 * kT, *ru = red + 4 * kT, *rdd = red + 6 * kT;
+    float *rxu = red, *rk = red + 4 * kT, *ru = red + 8 * kT, *rdd = red + 12 * kT;
     if ((lane & 3) == 0) {
-        rxu[ch * kT + rlo] = xu[0];
-        rxu[ch * kT + rhi] = xu[1];
-        rk[ch * kT + rlo] = kpart[0];
-        rk[ch * kT + rhi] = kpart[1];
-        ru[ch * kT + rlo] = upart[0];
-        ru[ch * kT + rhi] = upart[1];
+        rxu[cq * kT + rlo] = xu[0];
+        rxu[cq * kT + rhi] = xu[1];
+        rk[cq * kT + rlo] = kpart[0];
+        rk[cq * kT + rhi] = kpart[1];
+        ru[cq * kT + rlo] = upart[0];
+        ru[cq * kT + rhi] = upart[1];
     }
     if (lane == 0) rdd[warp] = dd;
     __syncthreads();
     if (tid < nr) {
-        ddt_dir[lb + r0 + tid] = rxu[tid] + rxu[kT + tid];
-        kq[lb + r0 + tid] = rk[tid] + rk[kT + tid];
-        uq[lb + r0 + tid] = ru[tid] + ru[kT + tid];
+        ddt_dir[lb + r0 + tid] = rxu[tid] + rxu[kT + tid] + rxu[2 * kT + tid] + rxu[3 * kT + tid];
+        kq[lb + r0 + tid] = rk[tid] + rk[kT + tid] + rk[2 * kT + tid] + rk[3 * kT + tid];
+        uq[lb + r0 + tid] = ru[tid] + ru[kT + tid] + ru[2 * kT + tid] + ru[3 * kT + tid];
     }
     if (tid == 0) {
         float sacc = 0.f;
-        for (int w = 0; w < 8; ++w) sacc += rdd[w];
+        for (int w = 0; w < kThr2 / 32; ++w) sacc += rdd[w];
         dDpart[(bh * nc + c) * nrt + rt] = sacc;
     }
 }
 
 // ---- tokens as targets --------------------------------------------------------------
+// grid (nc * nrt, H, B); a tile of 64 tokens l per CTA, 16 warps; source tiles s <= l double-buffered.
 template <int P, int N>
-__global__ void __launch_bounds__(kThr, 1)
+__global__ void __launch_bounds__(kThr2, 1)
     k_bwd_dst_mma(const bf16 *__restrict__ x, const bf16 *__restrict__ Bm, const bf16 *__restrict__ Cm,
                   const bf16 *__restrict__ dy, const float *__restrict__ acs, const float *__restrict__ dtw,
                   const float *__restrict__ s_in, int64_t L, int H, int G, int Q, int nc, int nrt,
                   float *__restrict__ dC_acc, float *__restrict__ tq) {
     constexpr int LN = N + 8, LP = P + 8, LW = kT + 8;
-    constexpr int TV = N / 16;
+    constexpr int TV = N / 32;
+    static_assert(TV % 2 == 0, "column quarters are whole n16 pairs");
     extern __shared__ __align__(16) unsigned char smem[];
-    bf16 *co = reinterpret_cast<bf16 *>(smem);  // [64][LN]  C_l
-    bf16 *dl = co + kT * LN;                     // [64][LP]  dy_l
-    bf16 *bs = dl + kT * LP;                     // [64][LN]  B_s
-    bf16 *xs = bs + kT * LN;                     // [64][LP]  x_s
-    bf16 *w3 = xs + kT * LP;                     // [64][LW]  W3 [l][s]
-    bf16 *si = w3 + kT * LW;                     // [P][LN]   S_in
+    bf16 *co = reinterpret_cast<bf16 *>(smem);  // [64][LN]     C_l
+    bf16 *dl = co + kT * LN;                     // [64][LP]     dy_l
+    bf16 *bs = dl + kT * LP;                     // [2][64][LN]  B_s (double buffer)
+    bf16 *xs = bs + 2 * kT * LN;                 // [2][64][LP]  x_s
+    bf16 *w3 = xs + 2 * kT * LP;                 // [64][LW]     W3 [l][s]
+    bf16 *si = w3 + kT * LW;                     // [P][LN]      S_in
     float *al = reinterpret_cast<float *>(si + P * LN);  // [64]
-    float *as = al + kT;                                 // [64]
-    float *ds = as + kT;                                 // [64]
-    float *red = ds + kT;                                // [2][64]
+    float *as = al + kT;                                 // [2][64]
+    float *ds = as + 2 * kT;                             // [2][64]
+    float *red = ds + 2 * kT;                            // [4][64]
 
     const int c = blockIdx.x / nrt, r0 = (blockIdx.x % nrt) * kT;
     const int h = blockIdx.y, b = blockIdx.z, g = h / (H / G);
@@ -481,16 +494,28 @@ __global__ void __launch_bounds__(kThr, 1)
     const int q = (int)min((int64_t)Q, L - t0);
     if (r0 >= q) return;
     const int nr = min(kT, q - r0);
+    const int send = r0 + nr;  // source tokens s < send
     const int64_t bh = (int64_t)b * H + h, lb = (bh * nc + c) * Q;
-    load_rows<N>(co, Cm + (((int64_t)b * L + t0 + r0) * G + g) * N, (int64_t)G * N, nr, tid);
-    load_rows<P>(dl, dy + (((int64_t)b * L + t0 + r0) * H + h) * P, (int64_t)H * P, nr, tid);
-    load_state_bf16<P, N>(si, s_in + (bh * nc + c) * (int64_t)P * N, tid);
-    for (int i = tid; i < kT; i += kThr) al[i] = acs[lb + min(r0 + i, Q - 1)];
-    async_wait();
+    load_rows<N>(co, Cm + (((int64_t)b * L + t0 + r0) * G + g) * N, (int64_t)G * N, nr, tid, kThr2);
+    load_rows<P>(dl, dy + (((int64_t)b * L + t0 + r0) * H + h) * P, (int64_t)H * P, nr, tid, kThr2);
+    {
+        const int n0s = min(kT, q);
+        load_rows<N>(bs, Bm + (((int64_t)b * L + t0) * G + g) * N, (int64_t)G * N, n0s, tid, kThr2);
+        load_rows<P>(xs, x + (((int64_t)b * L + t0) * H + h) * P, (int64_t)H * P, n0s, tid, kThr2);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        for (int i = tid; i < kT; i += kThr2) {
+            al[i] = acs[lb + min(r0 + i, Q - 1)];
+            as[i] = acs[lb + min(i, Q - 1)];
+            ds[i] = i < n0s ? dtw[lb + i] : 0.f;
+        }
+    }
+    load_state_bf16<P, N>(si, s_in + (bh * nc + c) * (int64_t)P * N, tid, kThr2);
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();
 
-    const int rb = warp & 3, ch = warp >> 2, nv0 = ch * (N / 2);
-    const uint32_t cob = su32(co), dlb = su32(dl), bsb = su32(bs), xsb = su32(xs), w3b = su32(w3), sib = su32(si);
+    const int rb = warp & 3, cq = warp >> 2, nv0 = cq * (N / 4);
+    const uint32_t cob = su32(co), dlb = su32(dl), w3b = su32(w3), sib = su32(si);
+    (void)cob;
     float aw[TV][4];
 #pragma unroll
     for (int j = 0; j < TV; ++j)
@@ -533,56 +558,61 @@ __global__ void __launch_bounds__(kThr, 1)
             for (int o = 1; o < 4; o <<= 1) cw[hf] += __shfl_xor_sync(0xffffffffu, cw[hf], o);
         }
         if ((lane & 3) == 0) {
-            red[ch * kT + rlo] = cw[0];
-            red[ch * kT + rhi] = cw[1];
+            red[cq * kT + rlo] = cw[0];
+            red[cq * kT + rhi] = cw[1];
         }
         __syncthreads();
-        if (tid < nr) tq[lb + r0 + tid] = red[tid] + red[kT + tid];
+        if (tid < nr) tq[lb + r0 + tid] = red[tid] + red[kT + tid] + red[2 * kT + tid] + red[3 * kT + tid];
     }
-    const int wr = warp & 3, wc = (warp >> 2) * 32;
-    for (int s0 = 0; s0 < r0 + nr; s0 += kT) {
-        const int ns = min(kT, q - s0);
-        __syncthreads();
-        load_rows<N>(bs, Bm + (((int64_t)b * L + t0 + s0) * G + g) * N, (int64_t)G * N, ns, tid);
-        load_rows<P>(xs, x + (((int64_t)b * L + t0 + s0) * H + h) * P, (int64_t)H * P, ns, tid);
-        for (int i = tid; i < kT; i += kThr) {
-            as[i] = acs[lb + min(s0 + i, Q - 1)];
-            ds[i] = i < ns ? dtw[lb + s0 + i] : 0.f;
+    const int wc = cq * 16;  // this warp's 16 columns s of a W3 tile
+    int it = 0;
+    for (int s0 = 0; s0 < send; s0 += kT, ++it) {
+        const int cur = it & 1, ns = min(kT, q - s0);
+        bf16 *bsc = bs + cur * kT * LN, *xsc = xs + cur * kT * LP;
+        const float *asc = as + cur * kT, *dsc = ds + cur * kT;
+        const int s1 = s0 + kT;
+        if (s1 < send) {  // prefetch the next source tile
+            const int n1 = min(kT, q - s1);
+            load_rows<N>(bs + (cur ^ 1) * kT * LN, Bm + (((int64_t)b * L + t0 + s1) * G + g) * N, (int64_t)G * N, n1,
+                         tid, kThr2);
+            load_rows<P>(xs + (cur ^ 1) * kT * LP, x + (((int64_t)b * L + t0 + s1) * H + h) * P, (int64_t)H * P, n1,
+                         tid, kThr2);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            for (int i = tid; i < kT; i += kThr2) {
+                as[(cur ^ 1) * kT + i] = acs[lb + min(s1 + i, Q - 1)];
+                ds[(cur ^ 1) * kT + i] = i < n1 ? dtw[lb + s1 + i] : 0.f;
+            }
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
-        async_wait();
         __syncthreads();
-        float f3[4][4];
+        const uint32_t bsb = su32(bsc), xsb = su32(xsc);
+        float f3[2][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) f3[j][e] = 0.f;
-#pragma unroll 2
+#pragma unroll 4
         for (int k0 = 0; k0 < P; k0 += 16) {
-            uint32_t a[4];
-            ldsm4(a_mk(dlb, LP, 16 * wr, k0, lane), a);
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                uint32_t bb[4];
-                ldsm4(b_nk(xsb, LP, wc + 16 * jj, k0, lane), bb);
-                mma(f3[2 * jj], a, bb[0], bb[1]);
-                mma(f3[2 * jj + 1], a, bb[2], bb[3]);
-            }
+            uint32_t a[4], bb[4];
+            ldsm4(a_mk(dlb, LP, 16 * rb, k0, lane), a);
+            ldsm4(b_nk(xsb, LP, wc, k0, lane), bb);
+            mma(f3[0], a, bb[0], bb[1]);
+            mma(f3[1], a, bb[2], bb[3]);
         }
-        {
-            const int llo = 16 * wr + (lane >> 2);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int sc = wc + 8 * j + 2 * (lane & 3);
+        for (int j = 0; j < 2; ++j) {
+            const int sc = wc + 8 * j + 2 * (lane & 3);
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const int l = llo + 8 * hf;
-                    float d0 = 0.f, d1 = 0.f;
-                    if (l < nr) {
-                        if (sc < ns && s0 + sc <= r0 + l) d0 = __expf(al[l] - as[sc]) * ds[sc];
-                        if (sc + 1 < ns && s0 + sc + 1 <= r0 + l) d1 = __expf(al[l] - as[sc + 1]) * ds[sc + 1];
-                    }
-                    *reinterpret_cast<uint32_t *>(w3 + l * LW + sc) = pack2(f3[j][2 * hf] * d0, f3[j][2 * hf + 1] * d1);
+            for (int hf = 0; hf < 2; ++hf) {
+                const int l = rlo + 8 * hf;
+                float d0 = 0.f, d1 = 0.f;
+                if (l < nr) {
+                    if (sc < ns && s0 + sc <= r0 + l) d0 = __expf(al[l] - asc[sc]) * dsc[sc];
+                    if (sc + 1 < ns && s0 + sc + 1 <= r0 + l) d1 = __expf(al[l] - asc[sc + 1]) * dsc[sc + 1];
                 }
+                *reinterpret_cast<uint32_t *>(w3 + l * LW + sc) = pack2(f3[j][2 * hf] * d0, f3[j][2 * hf + 1] * d1);
             }
         }
         __syncthreads();
@@ -599,6 +629,7 @@ __global__ void __launch_bounds__(kThr, 1)
                 mma(aw[2 * jj + 1], a, bb[2], bb[3]);
             }
         }
+        __syncthreads();
     }
     // epilogue: dC (fp32 atomics, group sum)
 #pragma unroll
@@ -618,11 +649,11 @@ __global__ void __launch_bounds__(kThr, 1)
 
 size_t sums_smem(int P, int N) { return (size_t)kT * ((P + 8) + (N + 8)) * 2; }
 size_t src_smem(int P, int N) {
-    return (size_t)(2 * kT * (N + 8) + 2 * kT * (P + 8) + 2 * kT * (kT + 8) + P * (N + 8)) * 2 +
-           (size_t)(3 * kT + 6 * kT + 8) * 4;
+    return (size_t)(3 * kT * (N + 8) + 3 * kT * (P + 8) + 2 * kT * (kT + 8) + P * (N + 8)) * 2 +
+           (size_t)(4 * kT + 12 * kT + 16) * 4;
 }
 size_t dst_smem(int P, int N) {
-    return (size_t)(2 * kT * (N + 8) + 2 * kT * (P + 8) + kT * (kT + 8) + P * (N + 8)) * 2 + (size_t)(5 * kT) * 4;
+    return (size_t)(3 * kT * (N + 8) + 3 * kT * (P + 8) + kT * (kT + 8) + P * (N + 8)) * 2 + (size_t)(9 * kT) * 4;
 }
 
 template <int P, int N>
@@ -659,7 +690,7 @@ cudaError_t launch_src(const FwdProblem &p, const void *dy, const float *acs, co
     if ((e = cudaFuncSetAttribute(k_bwd_src_mma<P, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
         return e;
     dim3 grid((unsigned)(p.nc * nrt), (unsigned)p.H, (unsigned)p.B);
-    k_bwd_src_mma<P, N><<<grid, kThr, smem, s>>>(
+    k_bwd_src_mma<P, N><<<grid, kThr2, smem, s>>>(
         static_cast<const bf16 *>(p.x), static_cast<const bf16 *>(p.Bm), static_cast<const bf16 *>(p.Cm),
         static_cast<const bf16 *>(dy), acs, dtw, gend, p.D, p.L, (int)p.H, (int)p.G, (int)p.Q, (int)p.nc, nrt,
         static_cast<bf16 *>(dx), dB_acc, kq, rq, uq, ddt_dir, dDpart);
@@ -675,7 +706,7 @@ cudaError_t launch_dst(const FwdProblem &p, const void *dy, const float *acs, co
     if ((e = cudaFuncSetAttribute(k_bwd_dst_mma<P, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
         return e;
     dim3 grid((unsigned)(p.nc * nrt), (unsigned)p.H, (unsigned)p.B);
-    k_bwd_dst_mma<P, N><<<grid, kThr, smem, s>>>(static_cast<const bf16 *>(p.x), static_cast<const bf16 *>(p.Bm),
+    k_bwd_dst_mma<P, N><<<grid, kThr2, smem, s>>>(static_cast<const bf16 *>(p.x), static_cast<const bf16 *>(p.Bm),
                                                  static_cast<const bf16 *>(p.Cm), static_cast<const bf16 *>(dy), acs,
                                                  dtw, s_in, p.L, (int)p.H, (int)p.G, (int)p.Q, (int)p.nc, nrt, dC_acc,
                                                  tq);
@@ -683,7 +714,7 @@ cudaError_t launch_dst(const FwdProblem &p, const void *dy, const float *acs, co
 }
 
 // (P, N) pairs with a compiled instance
-#define SSD_MMA_SHAPES(X) X(32, 64) X(64, 64) X(64, 128) X(64, 256) X(128, 128)
+#define SSD_MMA_SHAPES(X) X(64, 64) X(64, 128) X(64, 256) X(128, 128)
 
 }  // namespace
 
