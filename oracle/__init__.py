@@ -24,6 +24,16 @@ Forms (each in fp64 on the already-rounded inputs, layouts as in the library):
                      state after every token; select_state keeps the state at the
                      accepted position: "distilling Llama into Mamba" write-up,
                      "推测解码".
+  conv_split         the Mamba-2 block's convolution step: causal depthwise
+                     convolution of the x, B, C channels of the input projection,
+                     SiLU, split; dt = softplus(dt_raw + bias): "A Visual Guide to
+                     Mamba and SSMs", "The Mamba Block" (convolution before the SSM).
+  gated_rmsnorm      y * silu(z), normalised by its root mean square over groups of
+                     channels, times a weight: SSD write-up, "张量并行" (grouped norm).
+  mamba2_mixer       input projection, conv_split, the SSD recurrence, gated norm,
+                     output projection, in that order (Mamba-2 "parallel projection"
+                     block, SSD write-up "张量并行" and the Bi-Mamba summary's list of
+                     Mamba-2 layers).
   backward           the gradient of sum(dy * y) + sum(dh_final * h_final) with
                      respect to every input: the recurrence differentiated token
                      by token in reverse (C, OpenMP over (b, h)); the states are
@@ -236,3 +246,65 @@ def select_state(h0, states_out, accepted):
             raise ValueError("accepted index out of range")
         out[b] = h0[b] if a == 0 else states_out[b, a - 1]
     return out
+
+
+# ---- the Mamba-2 block around the SSD layer ---------------------------------------------
+
+def silu(v):
+    return v / (1.0 + np.exp(-v))
+
+
+def softplus(v):
+    return np.log1p(np.exp(-np.abs(v))) + np.maximum(v, 0.0)
+
+
+def conv_split(xbc, dt_raw, conv_w, conv_b, dt_bias, *, nheads, headdim, ngroups, dstate):
+    """Causal depthwise convolution over tokens of each of the Cc = H*P + 2*G*N channels of xbc
+    [B, L, Cc] with taps conv_w [Cc, W] (tap W-1 on the current token, inputs before the first
+    token are zero), plus conv_b [Cc] (or None), then SiLU; split into x [B,L,H,P], B, C
+    [B,L,G,N]. dt = softplus(dt_raw + dt_bias) [B,L,H]. Written as the sum over taps."""
+    xbc, dt_raw, conv_w, conv_b, dt_bias = map(_f64, (xbc, dt_raw, conv_w, conv_b, dt_bias))
+    Bsz, L, Cc = xbc.shape
+    W = conv_w.shape[1]
+    H, P, G, N = nheads, headdim, ngroups, dstate
+    assert Cc == H * P + 2 * G * N and dt_raw.shape == (Bsz, L, H)
+    acc = np.zeros_like(xbc) if conv_b is None else np.broadcast_to(conv_b, xbc.shape).copy()
+    for j in range(W):
+        shift = W - 1 - j  # tap j reads token t - shift
+        if shift == 0:
+            acc += conv_w[:, j] * xbc
+        elif shift < L:
+            acc[:, shift:, :] += conv_w[:, j] * xbc[:, :L - shift, :]
+    act = silu(acc)
+    x = act[..., :H * P].reshape(Bsz, L, H, P)
+    Bm = act[..., H * P:H * P + G * N].reshape(Bsz, L, G, N)
+    Cm = act[..., H * P + G * N:].reshape(Bsz, L, G, N)
+    dt = softplus(dt_raw + (0.0 if dt_bias is None else dt_bias))
+    return x, Bm, Cm, dt
+
+
+def gated_rmsnorm(y, z, weight, *, ngroups, eps):
+    """g = y * silu(z); per group of dim / ngroups consecutive channels,
+    out = weight * g / sqrt(mean(g^2) + eps). y, z [..., dim]."""
+    y, z, weight = map(_f64, (y, z, weight))
+    dim = y.shape[-1]
+    g = y * silu(z)
+    gg = g.reshape(*g.shape[:-1], ngroups, dim // ngroups)
+    r = 1.0 / np.sqrt(np.mean(gg * gg, axis=-1, keepdims=True) + eps)
+    return (gg * r).reshape(g.shape) * weight
+
+
+def mamba2_mixer(u, in_proj_w, conv_w, conv_b, dt_bias, A, D, norm_w, out_proj_w, *, nheads, headdim, ngroups,
+                 dstate, norm_groups, eps, h0=None):
+    """The Mamba-2 mixer forward. u [B, L, d_model]; in_proj_w [2*H*P + 2*G*N + H, d_model] gives
+    each token's row [z | x B C | dt_raw]; out_proj_w [d_model, H*P]. Returns (out, h_final)."""
+    u, in_proj_w, out_proj_w = map(_f64, (u, in_proj_w, out_proj_w))
+    H, P, G, N = nheads, headdim, ngroups, dstate
+    HP, GN = H * P, G * N
+    zxbcdt = u @ in_proj_w.T
+    z, xbc, dt_raw = zxbcdt[..., :HP], zxbcdt[..., HP:2 * HP + 2 * GN], zxbcdt[..., 2 * HP + 2 * GN:]
+    x, Bm, Cm, dt = conv_split(xbc, dt_raw, conv_w, conv_b, dt_bias, nheads=H, headdim=P, ngroups=G, dstate=N)
+    y, hf = recurrent(x, dt, A, Bm, Cm, D, h0)
+    o = gated_rmsnorm(y.reshape(*y.shape[:2], HP), z, norm_w, ngroups=norm_groups, eps=eps)
+    return o @ out_proj_w.T, hf
+
