@@ -499,6 +499,89 @@ def bwd_main(args, wl):
     return 0
 
 
+def block_main(args):
+    """The Mamba-2 mixer forward at the 2.7B-like layer (d_model 2560, H80 P64 N128 G1, conv
+    width 4, one norm group) on B4 L8192: in_proj GEMM (cuBLAS), ssd_conv_split, ssd_fwd,
+    ssd_gated_rmsnorm, out_proj GEMM (cuBLAS). One JSON line per part (CUDA events over --steps
+    calls of that part alone, each against its own roofline) and one for the whole mixer."""
+    import torch
+
+    from state_space_sequence_chunked_b200 import _binding as ssd
+    from state_space_sequence_chunked_b200 import inputs, mamba2
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    hbm, tf, src = peaks()
+    steps = max(args.steps, 1)
+    cfg = mamba2.MixerConfig(d_model=2560, nheads=80, headdim=64, ngroups=1, dstate=128, norm_groups=1)
+    Bsz, L = 4, 8192
+    d = inputs.draw_mixer(batch=Bsz, seqlen=L, d_model=cfg.d_model, nheads=cfg.nheads, headdim=cfg.headdim,
+                          ngroups=cfg.ngroups, dstate=cfg.dstate, seed=2)
+    g = {k: v.torch(dev) for k, v in d.items()}
+    w = mamba2.MixerWeights(in_proj=g["in_proj"], conv_w=g["conv_w"], conv_b=g["conv_b"], dt_bias=g["dt_bias"],
+                            A=g["A"], D=g["D"], norm_w=g["norm_w"], out_proj=g["out_proj"])
+    HP, GN, H, dm, Dp = cfg.d_inner, cfg.ngroups * cfg.dstate, cfg.nheads, cfg.d_model, cfg.d_in_proj
+    Cc = HP + 2 * GN
+    T = Bsz * L
+    zx = torch.matmul(g["u"], w.in_proj.t())
+    sp = ssd.ssd_conv_split(zx[..., HP:HP + Cc], zx[..., HP + Cc:], w.conv_w, w.conv_b, w.dt_bias, nheads=H,
+                            headdim=cfg.headdim, ngroups=cfg.ngroups, dstate=cfg.dstate)
+    y, hf = ssd.ssd_fwd(sp["x"], sp["dt"], w.A, sp["B"], sp["C"], w.D, None, chunk=cfg.chunk)
+    o = ssd.ssd_gated_rmsnorm(y.view(Bsz, L, HP), zx[..., :HP], w.norm_w, ngroups=1)
+    ws = torch.empty(max(ssd.fwd_workspace_bytes(Bsz, L, H, cfg.headdim, cfg.ngroups, cfg.dstate, ssd.SSD_BF16,
+                                                 cfg.chunk), 16), dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    parts = []
+
+    def part(name, fn, nbytes=0.0, flops=0.0):
+        ms = timed(fn)
+        t_b, t_f = nbytes / (hbm * 1e9), flops / (tf * 1e12)
+        bound = "tensor" if t_f > t_b else "hbm"
+        line = {"part": name, "ms": ms, "alg_bytes": nbytes, "alg_flops": flops, "bound": bound,
+                "frac": max(t_b, t_f) / (ms * 1e-3), "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+                "achieved_tflops": flops / (ms * 1e-3) / 1e12, "roofline_ms": max(t_b, t_f) * 1e3}
+        parts.append(line)
+        print(json.dumps(line), flush=True)
+
+    part("in_proj GEMM (cuBLAS)", lambda: torch.matmul(g["u"], w.in_proj.t(), out=zx),
+         2 * (T * dm + Dp * dm + T * Dp), 2.0 * T * dm * Dp)
+    part("ssd_conv_split", lambda: ssd.ssd_conv_split(zx[..., HP:HP + Cc], zx[..., HP + Cc:], w.conv_w, w.conv_b,
+                                                      w.dt_bias, nheads=H, headdim=cfg.headdim, ngroups=cfg.ngroups,
+                                                      dstate=cfg.dstate, out=sp, stream=stream),
+         2 * 2 * T * (Cc + H) + Cc * 4 * 5 + H * 4)
+    nb, fl = algorithmic(inputs.Workload("mixer", Bsz, L, H, cfg.headdim, cfg.dstate, cfg.ngroups, cfg.chunk, "bf16",
+                                         0.0, 2))
+    part("ssd_fwd", lambda: ssd.ssd_fwd(sp["x"], sp["dt"], w.A, sp["B"], sp["C"], w.D, None, chunk=cfg.chunk, y=y,
+                                        h_final=hf, workspace=ws, stream=stream), nb, fl)
+    part("ssd_gated_rmsnorm", lambda: ssd.ssd_gated_rmsnorm(y.view(Bsz, L, HP), zx[..., :HP], w.norm_w, ngroups=1,
+                                                            out=o, stream=stream), 3 * 2 * T * HP + HP * 4)
+    out = torch.empty(Bsz, L, dm, dtype=torch.bfloat16, device=dev)
+    part("out_proj GEMM (cuBLAS)", lambda: torch.matmul(o, w.out_proj.t(), out=out), 2 * (T * HP + dm * HP + T * dm),
+         2.0 * T * HP * dm)
+    ms = timed(lambda: mamba2.mixer_fwd(g["u"], w, cfg, stream=stream))
+    roof = sum(p_["roofline_ms"] for p_ in parts)
+    print(json.dumps({"metric": "Mamba-2 mixer fwd tokens/s at the 2.7B-like layer", "value": T / (ms * 1e-3),
+                      "unit": "tokens/s", "ms": ms, "sum_of_parts_ms": sum(p_["ms"] for p_ in parts),
+                      "roofline_ms": roof, "frac_of_roofline_time": roof / ms, "steps": steps,
+                      "config": {"batch": Bsz, "seqlen": L, "d_model": dm, "nheads": H, "headdim": cfg.headdim,
+                                 "dstate": cfg.dstate, "ngroups": cfg.ngroups, "conv_width": cfg.conv_width,
+                                 "norm_groups": 1, "dtype": "bf16"}, "peak_source": src}), flush=True)
+    return 0
+
+
 def aux_main(args):
     """Per-kernel timings of the kernels beside the forward, each against the HBM roofline
     (all of them are bandwidth-bound): the two verify flows on the spec-decode workload
@@ -605,6 +688,8 @@ def main():
     ap.add_argument("--workload", default="mamba2_2p7b")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block", action="store_true",
+                    help="time the Mamba-2 mixer forward around the SSD layer (1 GPU, one line per part)")
     ap.add_argument("--bwd", action="store_true",
                     help="time the backward pass (ssd_bwd) of the forward workload instead")
     ap.add_argument("--aux", action="store_true",
@@ -612,6 +697,8 @@ def main():
     args = ap.parse_args()
     if args.aux:
         return aux_main(args)
+    if args.block:
+        return block_main(args)
 
     from state_space_sequence_chunked_b200 import inputs
 

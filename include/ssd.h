@@ -310,6 +310,47 @@ ssd_status_t ssd_bwd(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *x,
                      float *dA, void *dBm, void *dCm, float *dD, float *dh0, void *workspace,
                      size_t workspace_bytes, void *stream);
 
+/*
+ * The Mamba-2 block around the SSD layer. The block's input projection (a plain GEMM) writes,
+ * per token, one row [z | x B C | dt_raw]; the SSD layer runs on x, B, C, dt; the gated,
+ * grouped norm of its output feeds the output projection (a plain GEMM). The pages describe
+ * the block in words only ("A Visual Guide to Mamba and SSMs", "The Mamba Block": an input
+ * projection, then a convolution before the SSM so tokens are not computed independently; the
+ * SSD write-up, "张量并行": every SSM parameter is a projection of the layer input, and the norm
+ * is grouped). These two calls are the operations between the GEMMs and ssd_fwd.
+ *
+ * ssd_conv_split: causal depthwise convolution of the x, B, C channels, SiLU, split into the
+ * layouts ssd_fwd takes, and the step size:
+ *   out[t, c] = silu(conv_b[c] + sum_{j<W} conv_w[c, j] * xbc[t - (W - 1) + j, c])  (zeros before t = 0)
+ *   channels c in [0, H*P) -> x [B,L,H,P]; [H*P, H*P + G*N) -> Bm [B,L,G,N]; the next G*N -> Cm
+ *   dt[b, t, h] = softplus(dt_raw[b, t, h] + dt_bias[h])
+ *   xbc      [B, L, *] dtype, row stride xbc_stride elements (>= H*P + 2*G*N, even), the
+ *            Cc = H*P + 2*G*N conv channels at the start of each row; 4-byte (bf16) or
+ *            8-byte (fp32) aligned
+ *   dt_raw   [B, L, *] dtype, row stride dt_stride (>= H), H values per row
+ *   conv_w   [Cc, W] fp32, 1 <= W <= 4; conv_b [Cc] fp32 or NULL (= 0); dt_bias [H] fp32 or NULL
+ *   x, Bm, Cm, dt   outputs, 16-byte aligned
+ * Requires H*P and G*N even. shape->... as in ssd_fwd.
+ */
+ssd_status_t ssd_conv_split(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *xbc, int64_t xbc_stride,
+                            const void *dt_raw, int64_t dt_stride, const float *conv_w, const float *conv_b,
+                            int64_t width, const float *dt_bias, void *x, void *Bm, void *Cm, void *dt,
+                            void *stream);
+
+/*
+ * ssd_gated_rmsnorm: for each of `rows` rows of `dim` channels, in `ngroups` groups of
+ * dim / ngroups consecutive channels,
+ *   g = y * silu(z),   out = weight * g / sqrt(mean over the group of g^2 + eps)
+ *   y      [rows, dim] dtype, contiguous, 16-byte aligned
+ *   z      [rows, *] dtype, row stride z_stride (>= dim, even), pair aligned (the z columns
+ *          of the input projection's rows can be passed in place)
+ *   weight [dim] fp32; out [rows, dim] dtype, 16-byte aligned
+ * Requires dim <= 8192, 1 <= ngroups <= 64 and (dim / ngroups) % 64 == 0.
+ */
+ssd_status_t ssd_gated_rmsnorm(int64_t rows, int64_t dim, int64_t ngroups, ssd_dtype_t dtype, const void *y,
+                               const void *z, int64_t z_stride, const float *weight, float eps, void *out,
+                               void *stream);
+
 #ifdef __cplusplus
 }
 #endif

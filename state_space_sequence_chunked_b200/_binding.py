@@ -52,6 +52,10 @@ _SIGS = {
     "ssd_cp_correct": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 8, ctypes.c_int),
     "ssd_bwd_workspace_bytes": ([ctypes.POINTER(ShapeT), ctypes.c_int, _i64, ctypes.POINTER(_sz)], ctypes.c_int),
     "ssd_bwd_plan": ([ctypes.POINTER(ShapeT), ctypes.c_int, _i64, ctypes.POINTER(PlanT)], ctypes.c_int),
+    "ssd_conv_split": ([ctypes.POINTER(ShapeT), ctypes.c_int, _vp, _i64, _vp, _i64, _vp, _vp, _i64] + [_vp] * 6,
+                       ctypes.c_int),
+    "ssd_gated_rmsnorm": ([_i64, _i64, _i64, ctypes.c_int, _vp, _vp, _i64, _vp, ctypes.c_float, _vp, _vp],
+                          ctypes.c_int),
     "ssd_bwd": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 7 + [_i64] + [_vp] * 9 + [_vp, _sz, _vp],
                 ctypes.c_int),
 }
@@ -101,6 +105,16 @@ def _dev(*ts):
             raise ValueError("libssd takes contiguous tensors")
         dev = t.device if dev is None else dev
     return dev
+
+
+def _dev_rows(dev, *ts):
+    """Row views (a column slice of wider rows): CUDA, on `dev`, unit column stride, rows at one
+    stride (the C calls take that stride)."""
+    for t in ts:
+        if not t.is_cuda or (dev is not None and t.device != dev):
+            raise ValueError("libssd takes CUDA tensors on one device")
+        if t.stride(-1) != 1 or any(t.stride(i) != t.stride(i + 1) * t.shape[i + 1] for i in range(t.dim() - 2)):
+            raise ValueError("row views need unit column stride and evenly spaced rows")
 
 
 def _stream(dev, stream):
@@ -306,3 +320,46 @@ def ssd_bwd(x, dt, A, B, C, D, h0, dy, dh_final=None, *, chunk: int, want_dD: bo
                        _stream(dev, stream))
     _check(st, "ssd_bwd")
     return o
+
+
+def ssd_conv_split(xbc, dt_raw, conv_w, conv_b, dt_bias, *, nheads, headdim, ngroups, dstate, out=None,
+                   stream=None):
+    """x [B,L,H,P], B, C [B,L,G,N], dt [B,L,H] from the convolution + SiLU of the x B C channels and
+    softplus(dt_raw + dt_bias). xbc and dt_raw are [B, L, *] views with unit column stride (the
+    input projection's columns can be passed in place)."""
+    dev = _dev(conv_w, conv_b, dt_bias)
+    _dev_rows(dev, xbc, dt_raw)
+    Bsz, L = xbc.shape[0], xbc.shape[1]
+    H, P, G, N = nheads, headdim, ngroups, dstate
+    assert xbc.stride(2) == 1 and dt_raw.stride(2) == 1 and xbc.stride(0) == L * xbc.stride(1)
+    assert dt_raw.stride(0) == L * dt_raw.stride(1)
+    code = _dtype_code(xbc)
+    o = dict(out or {})
+    o.setdefault("x", torch.empty(Bsz, L, H, P, dtype=xbc.dtype, device=dev))
+    o.setdefault("B", torch.empty(Bsz, L, G, N, dtype=xbc.dtype, device=dev))
+    o.setdefault("C", torch.empty(Bsz, L, G, N, dtype=xbc.dtype, device=dev))
+    o.setdefault("dt", torch.empty(Bsz, L, H, dtype=xbc.dtype, device=dev))
+    shape = ShapeT(Bsz, L, H, P, G, N)
+    st = lib().ssd_conv_split(ctypes.byref(shape), code, _ptr(xbc), xbc.stride(1), _ptr(dt_raw), dt_raw.stride(1),
+                              _ptr(conv_w), _ptr(conv_b), conv_w.shape[1], _ptr(dt_bias), _ptr(o["x"]), _ptr(o["B"]),
+                              _ptr(o["C"]), _ptr(o["dt"]), _stream(dev, stream))
+    _check(st, "ssd_conv_split")
+    return o
+
+
+def ssd_gated_rmsnorm(y, z, weight, *, ngroups, eps=1e-5, out=None, stream=None):
+    """out = weight * RMSNorm over `ngroups` groups of (y * silu(z)); y [..., dim] contiguous,
+    z [..., dim] with unit column stride (a column slice of a wider row is fine)."""
+    dev = _dev(y, weight, out)
+    _dev_rows(dev, z)
+    dim = y.shape[-1]
+    rows = y.numel() // dim if dim else 0
+    assert z.stride(-1) == 1
+    zs = z.stride(-2) if z.dim() >= 2 else dim
+    if out is None:
+        out = torch.empty_like(y)
+    st = lib().ssd_gated_rmsnorm(rows, dim, ngroups, _dtype_code(y), _ptr(y), _ptr(z), zs, _ptr(weight), float(eps),
+                                 _ptr(out), _stream(dev, stream))
+    _check(st, "ssd_gated_rmsnorm")
+    return out
+

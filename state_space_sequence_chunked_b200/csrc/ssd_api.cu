@@ -342,3 +342,47 @@ SSD_API ssd_status_t ssd_bwd(const ssd_shape_t *shape, ssd_dtype_t dtype, const 
     const BwdGrads g{dy, dh_final, dx, ddt, dBm, dCm, dA, dD, dh0};
     return from_cuda(simt_bwd(p, g, workspace, s));
 }
+
+SSD_API ssd_status_t ssd_conv_split(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *xbc, int64_t xbc_stride,
+                                    const void *dt_raw, int64_t dt_stride, const float *conv_w, const float *conv_b,
+                                    int64_t width, const float *dt_bias, void *x, void *Bm, void *Cm, void *dt,
+                                    void *stream) {
+    ssd_status_t st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if ((st = check_dtype(dtype)) != SSD_OK) return st;
+    const int64_t HP = shape->nheads * shape->headdim, GN = shape->ngroups * shape->dstate;
+    if (width < 1 || width > 4 || xbc_stride < HP + 2 * GN || dt_stride < shape->nheads) return SSD_ERR_INVALID_ARG;
+    if (HP % 2 != 0 || GN % 2 != 0 || xbc_stride % 2 != 0) return SSD_ERR_UNSUPPORTED;
+    if (shape->batch == 0 || shape->seqlen == 0) return SSD_OK;
+    if (!xbc || !dt_raw || !conv_w || !x || !Bm || !Cm || !dt) return SSD_ERR_INVALID_ARG;
+    const uintptr_t pair = dtype == SSD_F32 ? 8 : 4, elem = dtype == SSD_F32 ? 4 : 2;
+    if ((reinterpret_cast<uintptr_t>(xbc) & (pair - 1)) || (reinterpret_cast<uintptr_t>(dt_raw) & (elem - 1)))
+        return SSD_ERR_ALIGNMENT;
+    const void *ptrs[] = {conv_w, conv_b, dt_bias, x, Bm, Cm, dt};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return SSD_ERR_ALIGNMENT;
+    const BlockShape s{shape->batch, shape->seqlen, shape->nheads, shape->headdim, shape->ngroups, shape->dstate};
+    return from_cuda(conv_split_launch(s, dtype, xbc, xbc_stride, dt_raw, dt_stride, conv_w, conv_b, (int)width,
+                                       dt_bias, x, Bm, Cm, dt, static_cast<cudaStream_t>(stream)));
+}
+
+SSD_API ssd_status_t ssd_gated_rmsnorm(int64_t rows, int64_t dim, int64_t ngroups, ssd_dtype_t dtype, const void *y,
+                                       const void *z, int64_t z_stride, const float *weight, float eps, void *out,
+                                       void *stream) {
+    ssd_status_t st = check_dtype(dtype);
+    if (st != SSD_OK) return st;
+    if (rows < 0 || dim < 1 || ngroups < 1 || dim % ngroups != 0 || z_stride < dim || !(eps >= 0.f))
+        return SSD_ERR_INVALID_ARG;
+    if (dim > gated_rmsnorm_max_dim() || ngroups > 64 || (dim / ngroups) % 64 != 0 || z_stride % 2 != 0 ||
+        rows > 0x7fffffffLL)
+        return SSD_ERR_UNSUPPORTED;
+    if (rows == 0) return SSD_OK;
+    if (!y || !z || !weight || !out) return SSD_ERR_INVALID_ARG;
+    const uintptr_t pair = dtype == SSD_F32 ? 8 : 4;
+    if (reinterpret_cast<uintptr_t>(z) & (pair - 1)) return SSD_ERR_ALIGNMENT;
+    const void *ptrs[] = {y, weight, out};
+    for (const void *q : ptrs)
+        if (!aligned16(q)) return SSD_ERR_ALIGNMENT;
+    return from_cuda(gated_rmsnorm_launch(rows, (int)dim, (int)ngroups, dtype, y, z, z_stride, weight, eps, out,
+                                          static_cast<cudaStream_t>(stream)));
+}

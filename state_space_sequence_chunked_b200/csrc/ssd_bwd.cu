@@ -90,6 +90,7 @@ __global__ void __launch_bounds__(kThreads)
     const int h = blockIdx.y, b = blockIdx.z;
     const int64_t bh = (int64_t)b * H + h;
     const bool valid = e < PN;
+    __shared__ float red[8][kThreads / 32];
     float run = (valid && dh_final) ? dh_final[bh * PN + e] : 0.f;
     if (dh_final) {
         const float part = warp_sum(valid ? run * hfin[bh * PN + e] : 0.f);
@@ -97,25 +98,37 @@ __global__ void __launch_bounds__(kThreads)
     }
     // serial in c; the loads of 8 chunks are issued before the chain
     for (int c1 = nc - 1; c1 >= 0; c1 -= 8) {
-        float r[8], dec[8], si[8];
+        float r[8], dec[8], si[8], part[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int c = c1 - i;
             r[i] = (valid && c >= 0) ? dstates[(bh * nc + c) * PN + e] : 0.f;
             si[i] = (ec && valid && c >= 0) ? s_in[(bh * nc + c) * PN + e] : 0.f;
             dec[i] = c >= 0 ? acs[(bh * nc + c) * Q + Q - 1] : 0.f;
+            part[i] = 0.f;
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int c = c1 - i;
             if (c >= 0) {
                 if (valid) dstates[(bh * nc + c) * PN + e] = run;
-                if (ec) {
-                    const float part = warp_sum(run * si[i]);
-                    if ((threadIdx.x & 31) == 0) atomicAdd(ec + bh * nc + c, part);
-                }
+                if (ec) part[i] = run * si[i];
                 run = fmaf(expf(dec[i]), run, r[i]);
             }
+        }
+        if (ec) {  // <Gend[c], S_in[c]>: reduced over the CTA, then one atomic per chunk
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float v = warp_sum(part[i]);
+                if ((threadIdx.x & 31) == 0) red[i][threadIdx.x >> 5] = v;
+            }
+            __syncthreads();
+            if (threadIdx.x < 8 && c1 - (int)threadIdx.x >= 0) {
+                float v = 0.f;
+                for (int w = 0; w < kThreads / 32; ++w) v += red[threadIdx.x][w];
+                atomicAdd(ec + bh * nc + c1 - threadIdx.x, v);
+            }
+            __syncthreads();
         }
     }
     if (valid && dh0) dh0[bh * PN + e] = run;

@@ -105,6 +105,17 @@ cudaError_t cp_correct_tc_launch(const CpProblem &p, const void *dt, const float
 cudaError_t cp_correct_launch(const CpProblem &p, const void *dt, const float *A, const void *Cm, const float *bsum,
                               const float *s_in, void *y, int *status, cudaStream_t s);
 
+// ---- the Mamba-2 block around the SSD: conv + split, gated grouped RMSNorm ------------
+struct BlockShape {
+    int64_t B, L, H, P, G, N;
+};
+cudaError_t conv_split_launch(const BlockShape &s, ssd_dtype_t dtype, const void *xbc, int64_t xbc_stride,
+                              const void *dt_raw, int64_t dt_stride, const float *conv_w, const float *conv_b,
+                              int width, const float *dt_bias, void *x, void *Bm, void *Cm, void *dt, cudaStream_t st);
+int gated_rmsnorm_max_dim();
+cudaError_t gated_rmsnorm_launch(int64_t rows, int dim, int ngroups, ssd_dtype_t dtype, const void *y, const void *z,
+                                 int64_t z_stride, const float *w, float eps, void *out, cudaStream_t st);
+
 // ---- element access ---------------------------------------------------------------
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }

@@ -155,3 +155,26 @@ def draw_cotangents(wl: Workload, *, batch=None, seqlen=None, seed=None, dh_std=
     dy = rng.standard_normal((Bsz, L, H, P))
     dhf = rng.standard_normal((Bsz, H, P, N)) * dh_std if dh_std > 0 else None
     return {"dy": Tensor(dy, wl.dtype), "dh_final": Tensor(dhf, "f32") if dhf is not None else None}
+
+
+def draw_mixer(*, batch, seqlen, d_model, nheads, headdim, ngroups, dstate, conv_width=4, dtype="bf16", seed=0):
+    """Input and random-init weights of one Mamba-2 mixer (no trained weights exist here).
+    u ~ N(0, 1) [B, L, d_model]; in_proj ~ N(0, 1/d_model) [2HP + 2GN + H, d_model] and
+    out_proj ~ N(0, 1/HP) [d_model, HP] in the storage dtype; fp32 conv taps ~ N(0, 1/W), conv
+    bias ~ N(0, 0.01), dt bias ~ U(-7, -2.3) (softplus of it lies near [1e-3, 1e-1]),
+    A = -exp(U(0, ln 16)), D ~ N(0, 1), norm weight ~ 1 + N(0, 0.01)."""
+    HP, GN = nheads * headdim, ngroups * dstate
+    Dp, Cc = 2 * HP + 2 * GN + nheads, HP + 2 * GN
+    rng = np.random.default_rng(seed)
+    out = {
+        "u": Tensor(rng.standard_normal((batch, seqlen, d_model)), dtype),
+        "in_proj": Tensor(rng.standard_normal((Dp, d_model)) / math.sqrt(d_model), dtype),
+        "conv_w": Tensor(rng.standard_normal((Cc, conv_width)) / math.sqrt(conv_width), "f32"),
+        "conv_b": Tensor(rng.standard_normal(Cc) * 0.1, "f32"),
+        "dt_bias": Tensor(rng.uniform(-7.0, -2.3, size=nheads), "f32"),
+        "A": Tensor(-np.exp(rng.uniform(0.0, math.log(16.0), size=nheads)), "f32"),
+        "D": Tensor(rng.standard_normal(nheads), "f32"),
+        "norm_w": Tensor(1.0 + 0.1 * rng.standard_normal(HP), "f32"),
+        "out_proj": Tensor(rng.standard_normal((d_model, HP)) / math.sqrt(HP), dtype),
+    }
+    return out

@@ -34,7 +34,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("ssd_fwd", "ssd_verify", "ssd_select_state", "ssd_fwd_workspace_bytes", "ssd_strerror",
               "ssd_advance_state", "ssd_decode_step", "ssd_cp_decay", "ssd_cp_combine", "ssd_cp_correct",
-              "ssd_bwd", "ssd_bwd_workspace_bytes"):
+              "ssd_bwd", "ssd_bwd_workspace_bytes", "ssd_conv_split", "ssd_gated_rmsnorm"):
         assert n in names
 
 
@@ -135,6 +135,36 @@ def test_bwd_workspace_bytes(lib):
     assert out.value == 0
     assert lib.ssd_bwd_workspace_bytes(ctypes.byref(shp), 1, 256, None) == 1
     assert lib.ssd_bwd_workspace_bytes(ctypes.byref(B.ShapeT(1, 10, 4, 16, 3, 16)), 1, 64, ctypes.byref(out)) == 1
+
+
+def test_block_ops_reject_before_launch(lib):
+    shp = B.ShapeT(2, 100, 4, 16, 1, 8)
+    vp = ctypes.c_void_p
+    good = dict(xbc=0x10000, dtr=0x20000, w=0x30000, b=None, dtb=None, x=0x40000, Bm=0x50000, Cm=0x60000, dt=0x70000)
+
+    def conv(p=good, stride=96, dstride=100, width=4, shape=shp, dtype=B.SSD_BF16):
+        q = {k: vp(v) if v else None for k, v in p.items()}
+        return lib.ssd_conv_split(ctypes.byref(shape), dtype, q["xbc"], stride, q["dtr"], dstride, q["w"], q["b"],
+                                  width, q["dtb"], q["x"], q["Bm"], q["Cm"], q["dt"], None)
+    for k in ("xbc", "dtr", "w", "x", "Bm", "Cm", "dt"):
+        assert conv({**good, k: None}) == 1, k
+    assert conv(width=0) == 1 and conv(width=5) == 1
+    assert conv(stride=79) == 1        # < H*P + 2*G*N = 80
+    assert conv(stride=97) == 2        # odd row stride
+    assert conv(dstride=3) == 1        # < H
+    assert conv({**good, "xbc": 0x10002}) == 3 and conv({**good, "x": 0x40004}) == 3
+    assert conv(shape=B.ShapeT(2, 100, 3, 5, 1, 8)) == 2  # H*P odd
+
+    def norm(rows=10, dim=256, ng=4, y=0x10000, z=0x20000, zs=256, w=0x30000, eps=1e-5, out=0x40000):
+        return lib.ssd_gated_rmsnorm(rows, dim, ng, B.SSD_BF16, vp(y) if y else None, vp(z) if z else None, zs,
+                                     vp(w) if w else None, ctypes.c_float(eps), vp(out) if out else None, None)
+    assert norm(y=None) == 1 and norm(w=None) == 1 and norm(out=None) == 1
+    assert norm(dim=250, ng=5) == 2          # group of 50 channels
+    assert norm(dim=256, ng=3) == 1          # groups do not divide dim
+    assert norm(dim=8256, ng=1, zs=8256) == 2  # wider than the kernel's row
+    assert norm(zs=128) == 1 and norm(eps=-1.0) == 1
+    assert norm(z=0x20002) == 3 and norm(y=0x10004) == 3
+    assert norm(rows=0, y=None, z=None, w=None, out=None) == 0
 
 
 def test_bwd_plan_selects_path(lib):
