@@ -342,8 +342,9 @@ ssd_status_t ssd_conv_split(const ssd_shape_t *shape, ssd_dtype_t dtype, const v
  * dim / ngroups consecutive channels,
  *   g = y * silu(z),   out = weight * g / sqrt(mean over the group of g^2 + eps)
  *   y      [rows, dim] dtype, contiguous, 16-byte aligned
- *   z      [rows, *] dtype, row stride z_stride (>= dim, even), pair aligned (the z columns
- *          of the input projection's rows can be passed in place)
+ *   z      [rows, *] dtype, row stride z_stride (>= dim, even), 4-byte (bf16) or 8-byte (fp32)
+ *          aligned: the z columns of the input projection's rows can be passed in place (16-byte
+ *          aligned rows take 16-byte loads)
  *   weight [dim] fp32; out [rows, dim] dtype, 16-byte aligned
  * Requires dim <= 8192, 1 <= ngroups <= 64 and (dim / ngroups) % 64 == 0.
  */

@@ -164,6 +164,7 @@ def test_block_ops_reject_before_launch(lib):
     assert norm(dim=8256, ng=1, zs=8256) == 2  # wider than the kernel's row
     assert norm(zs=128) == 1 and norm(eps=-1.0) == 1
     assert norm(z=0x20002) == 3 and norm(y=0x10004) == 3
+    assert norm(zs=257) == 2                 # odd z row stride
     assert norm(rows=0, y=None, z=None, w=None, out=None) == 0
 
 

@@ -47,15 +47,16 @@ def test_conv_split(cuda_device, dtype, W, bias, L):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("dim,ngroups", [(256, 1), (512, 8), (5120, 1), (5120, 8), (8192, 64)])
-def test_gated_rmsnorm(cuda_device, dtype, dim, ngroups):
+@pytest.mark.parametrize("zoff,zpad", [(8, 16), (2, 10)])  # 16-byte aligned z rows, and not
+def test_gated_rmsnorm(cuda_device, dtype, dim, ngroups, zoff, zpad):
     rng = np.random.default_rng(dim + ngroups)
     rows = 37
     y = as_stored(rng.standard_normal((rows, dim)), dtype)
-    zrow = as_stored(rng.standard_normal((rows, dim + 10)), dtype)  # z: a column slice of wider rows
+    zrow = as_stored(rng.standard_normal((rows, dim + zpad)), dtype)  # z: a column slice of wider rows
     w = as_stored(1 + 0.1 * rng.standard_normal(dim), "f32")
-    ref = oracle.gated_rmsnorm(y, zrow[:, 4:4 + dim], w, ngroups=ngroups, eps=1e-5)
+    ref = oracle.gated_rmsnorm(y, zrow[:, zoff:zoff + dim], w, ngroups=ngroups, eps=1e-5)
     zt = torch.from_numpy(zrow).to(cuda_device, tdt(dtype))
-    out = ssd.ssd_gated_rmsnorm(torch.from_numpy(y).to(cuda_device, tdt(dtype)), zt[:, 4:4 + dim],
+    out = ssd.ssd_gated_rmsnorm(torch.from_numpy(y).to(cuda_device, tdt(dtype)), zt[:, zoff:zoff + dim],
                                 torch.from_numpy(w).float().to(cuda_device), ngroups=ngroups, eps=1e-5)
     torch.cuda.synchronize()
     assert rel_err(to_np(out), ref) <= TOL[dtype]
