@@ -144,7 +144,7 @@ __device__ __noinline__ void gprime_exact(uint32_t gaddr, int qtr, int row, floa
             uint32_t r[32];
             tmem_ld32(gaddr + 32 * jb, r);
             tmem_wait_ld(r);
-#pragma unroll 4
+#pragma unroll  // whole: r and out stay in registers
             for (int i = 0; i < 16; ++i) {
                 const int s = 32 * jb + 2 * i;
                 float v0 = s <= row ? __uint_as_float(r[2 * i]) * ex2(acs_r - acsW[s]) * dk[s] : 0.f;
