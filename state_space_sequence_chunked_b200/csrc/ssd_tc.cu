@@ -130,9 +130,10 @@ __device__ __forceinline__ Share share_of(long long total, int nc, int i, int G)
 // ---------------------------------------------------------------------------------
 
 // Exact form of G' for one warp's 32 rows (lane quarter qtr): every element of the causal
-// part takes its own exponential, D_h on the diagonal. Out of line: it runs only for blocks
-// whose decay range is too wide for the factored form.
-__device__ __noinline__ void gprime_exact(uint32_t gaddr, int qtr, int row, float acs_r, const float *acsW,
+// part takes its own exponential, D_h on the diagonal (blocks whose decay range is too wide
+// for the factored form). A_cs and dt come by explicit shared-memory loads, two columns at a
+// time; volatile, so that they stay after the barrier wait that makes those values valid.
+__device__ __forceinline__ void gprime_exact(uint32_t gaddr, int qtr, int row, float acs_r, const float *acsW,
                                           const float *dk, float Dh) {
 #pragma unroll 1
     for (int jb = 0; jb < 4; ++jb) {
@@ -144,11 +145,16 @@ __device__ __noinline__ void gprime_exact(uint32_t gaddr, int qtr, int row, floa
             uint32_t r[32];
             tmem_ld32(gaddr + 32 * jb, r);
             tmem_wait_ld(r);
+            const uint32_t aw = (uint32_t)__cvta_generic_to_shared(acsW + 32 * jb);
+            const uint32_t dw = (uint32_t)__cvta_generic_to_shared(dk + 32 * jb);
 #pragma unroll  // whole: r and out stay in registers
             for (int i = 0; i < 16; ++i) {
                 const int s = 32 * jb + 2 * i;
-                float v0 = s <= row ? __uint_as_float(r[2 * i]) * ex2(acs_r - acsW[s]) * dk[s] : 0.f;
-                float v1 = s + 1 <= row ? __uint_as_float(r[2 * i + 1]) * ex2(acs_r - acsW[s + 1]) * dk[s + 1] : 0.f;
+                float a0, a1, d0, d1;
+                asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(a0), "=f"(a1) : "r"(aw + 8 * i));
+                asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(d0), "=f"(d1) : "r"(dw + 8 * i));
+                float v0 = s <= row ? __uint_as_float(r[2 * i]) * ex2(acs_r - a0) * d0 : 0.f;
+                float v1 = s + 1 <= row ? __uint_as_float(r[2 * i + 1]) * ex2(acs_r - a1) * d1 : 0.f;
                 v0 += s == row ? Dh : 0.f;
                 v1 += s + 1 == row ? Dh : 0.f;
                 out[i] = pack_bf16(v0, v1);
