@@ -283,3 +283,24 @@ def test_binding_requires_cuda_tensors():
     x = torch.zeros(1, 4, 2, 8)
     with pytest.raises(ValueError):
         B.ssd_fwd(x, torch.zeros(1, 4, 2), torch.zeros(2), torch.zeros(1, 4, 1, 8), torch.zeros(1, 4, 1, 8), chunk=4)
+    # every other entry point refuses host tensors too: there is no CPU path
+    with pytest.raises(ValueError):
+        B.ssd_bwd(x, torch.zeros(1, 4, 2), torch.zeros(2), torch.zeros(1, 4, 1, 8), torch.zeros(1, 4, 1, 8), None,
+                  None, torch.zeros_like(x), chunk=4)
+    row = torch.zeros(1, 4, 2 * 16 + 2 * 8 + 2)
+    with pytest.raises(ValueError):
+        B.ssd_conv_split(row[..., 16:48], row[..., 48:50], torch.zeros(32, 4), None, None, nheads=2, headdim=8,
+                         ngroups=1, dstate=8)
+    with pytest.raises(ValueError):
+        B.ssd_gated_rmsnorm(torch.zeros(3, 64), torch.zeros(3, 64), torch.ones(64), ngroups=1)
+    with pytest.raises(ValueError):
+        B.ssd_verify(torch.zeros(1, 2, 8, 8), torch.zeros(1, 2, 2, 8), torch.zeros(1, 2, 2), torch.zeros(2),
+                     torch.zeros(1, 2, 1, 8), torch.zeros(1, 2, 1, 8))
+
+
+def test_mixer_config_sizes():
+    """The input projection's row holds z, x, B, C (H*P, H*P, G*N, G*N) and dt_raw (H)."""
+    from state_space_sequence_chunked_b200 import mamba2
+
+    cfg = mamba2.MixerConfig(d_model=2560, nheads=80, headdim=64, ngroups=1, dstate=128)
+    assert cfg.d_inner == 5120 and cfg.d_in_proj == 2 * 5120 + 2 * 128 + 80
