@@ -54,6 +54,8 @@ BF16_CASES = [
     (1, 1, 2, 64, 1, 128, 256, 0.1),       # a single token
     (1, 90, 2, 200, 1, 40, 32, 0.1),       # headdim and dstate not multiples of 32
     (1, 64, 2, 256, 1, 256, 64, 0.1),      # the largest tiles
+    (1, 300, 2, 64, 1, 128, 100, 0.1),     # tensor-core path, chunk not a multiple of the 64-token tile
+    (2, 130, 4, 64, 2, 64, 48, 0.0),       # tensor-core path, chunk below one tile, groups
 ]
 
 
