@@ -81,6 +81,10 @@ int mma_row_tiles(const FwdProblem &p);
 bool tc_supported(const FwdProblem &p);
 size_t tc_fwd_workspace_bytes(const FwdProblem &p);
 cudaError_t tc_fwd(const FwdProblem &p, void *ws, cudaStream_t s);
+// the two-heads-per-task kernel that tc_fwd runs where it applies (N = 128, heads per group even)
+bool tc_pair_supported(const FwdProblem &p);
+size_t tc_pair_workspace_bytes(const FwdProblem &p);
+cudaError_t tc_pair_fwd(const FwdProblem &p, void *ws, cudaStream_t s);
 
 // ---- verify / select --------------------------------------------------------------
 cudaError_t verify_launch(const VerifyProblem &p, cudaStream_t s);

@@ -798,11 +798,14 @@ static int tc_grid(const FwdProblem &p) {
 }
 
 size_t tc_fwd_workspace_bytes(const FwdProblem &p) {
+    if (tc_pair_supported(p)) return tc_pair_workspace_bytes(p);
     const size_t g = (size_t)tc_grid(p);
     return kWsAlign + align_up(g * sizeof(int), kWsAlign) + g * (size_t)(tc::kP * p.N) * sizeof(float);
 }
 
+// Two heads per task (C B^T shared) where the heads pair up within groups; one head otherwise.
 cudaError_t tc_fwd(const FwdProblem &p, void *ws, cudaStream_t s) {
+    if (tc_pair_supported(p)) return tc_pair_fwd(p, ws, s);
     const int grid = tc_grid(p);
     char *base = static_cast<char *>(ws);
     int *status = reinterpret_cast<int *>(base);

@@ -104,13 +104,16 @@ def _zeroed(d, *names):
     return d
 
 
+@pytest.mark.parametrize("nheads", [1, 2])
 @pytest.mark.parametrize("what", ["skip", "state_to_output", "diagonal_block", "all"])
-def test_tensor_core_products_in_isolation(cuda_device, what):
+def test_tensor_core_products_in_isolation(cuda_device, what, nheads):
     """One 128-token block with all but one product switched off, so a wrong
     operand layout shows up as exactly one failing case:
     skip: dt = 0, h0 = 0 -> y = D x;  state_to_output: dt = 0, x = 0, D = 0 -> y = C h0^T;
-    diagonal_block: h0 = 0, D = 0 -> y = (C B^T o L) (dt x), h_final = chunk state."""
-    d = _tc_case(7)
+    diagonal_block: h0 = 0, D = 0 -> y = (C B^T o L) (dt x), h_final = chunk state.
+    One head runs the one-head kernel, two heads the head-pair kernel (dt = 0 on valid
+    tokens sends a pair task to its single-head exact form)."""
+    d = _tc_case(7, nheads=nheads)
     zero = {"skip": ("dt", "h0"), "state_to_output": ("dt", "x", "D"), "diagonal_block": ("h0", "D"),
             "all": ()}[what]
     d = _zeroed(d, *zero)
