@@ -370,54 +370,71 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int4 cu = crd_raw;
             const int nvalid = nvalid_raw;
             const int h0i = 2 * cu.y;
-            bool fact = true;
-            float hd_lane = 0.f;  // field (lane & 7) of head (lane >> 3) of the two Head0 records
-#pragma unroll 1
-            for (int e = 0; e < 2; ++e) {
-                float d[4];
+            // Both heads in one pass: lanes 16 e .. 16 e + 15 take head e, lane g of the half
+            // tokens 8 g .. 8 g + 7 (from the pairs that lanes 2 g and 2 g + 1 fetched).
+            const int e = lane >> 4, g = lane & 15;
+            uint32_t hv[4];  // this lane's 8 dt of head e, bf16 pairs in token order
+            {
+                uint32_t p0[4], p1[4];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) d[m] = e == 0 ? bf16_lo(raw[m]) : bf16_hi(raw[m]);
-                const float a2 = __fmul_rn(__ldg(prm.A + h0i + e), kLog2e);
-                const float v0 = __fmul_rn(d[0], a2), v1 = __fmaf_rn(d[1], a2, v0), v2 = __fmaf_rn(d[2], a2, v1),
-                            v3 = __fmaf_rn(d[3], a2, v2);
-                float incl = v3;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float q = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl = __fadd_rn(incl, q);
+                for (int m = 0; m < 4; ++m) {
+                    p0[m] = __shfl_sync(0xffffffffu, raw[m], 2 * g);
+                    p1[m] = __shfl_sync(0xffffffffu, raw[m], 2 * g + 1);
                 }
-                const float excl = __fsub_rn(incl, v3);
-                const float a0 = __fadd_rn(excl, v0), a1 = __fadd_rn(excl, v1), a2v = __fadd_rn(excl, v2);
-                float mx = fmaxf(fmaxf(a0, a1), fmaxf(a2v, incl)), mn = fminf(fminf(a0, a1), fminf(a2v, incl));
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-                }
-                const int nv = nvalid - 4 * lane;
-                bool dt_ok = true;
-#pragma unroll
-                for (int m = 0; m < 4; ++m) dt_ok = dt_ok && (nv <= m || fabsf(d[m]) >= 0x1p-40f);
-                // (mx - mn <= 128 is false for NaN, which then takes the exact form)
-                fact = fact && __all_sync(0xffffffffu, dt_ok) && (mx - mn <= 128.f);
-                // Head0 = {m, tot, off1, off2, off3, a2, Dh, 0}; off q = the cumsum through token 32 q - 1
-                const float tot = __shfl_sync(0xffffffffu, incl, 31), off1 = __shfl_sync(0xffffffffu, incl, 7),
-                            off2 = __shfl_sync(0xffffffffu, incl, 15), off3 = __shfl_sync(0xffffffffu, incl, 23);
-                if ((lane >> 3) == e) {
-                    const int f = lane & 7;
-                    hd_lane = f == 0 ? __fmul_rn(0.5f, __fadd_rn(mx, mn))
-                                     : f == 1 ? tot
-                                     : f == 2 ? off1
-                                     : f == 3 ? off2
-                                     : f == 4 ? off3
-                                     : f == 5 ? a2
-                                     : f == 6 ? (prm.D ? __ldg(prm.D + h0i + e) : 0.f)
-                                              : 0.f;
-                }
+                // tokens 8 g + m from lane 2 g, 8 g + 4 + m from lane 2 g + 1; head e's half of each pair
+                const uint32_t sh16 = e ? 16u : 0u;
+                hv[0] = ((p0[0] >> sh16) & 0xFFFFu) | (((p0[1] >> sh16) & 0xFFFFu) << 16);
+                hv[1] = ((p0[2] >> sh16) & 0xFFFFu) | (((p0[3] >> sh16) & 0xFFFFu) << 16);
+                hv[2] = ((p1[0] >> sh16) & 0xFFFFu) | (((p1[1] >> sh16) & 0xFFFFu) << 16);
+                hv[3] = ((p1[2] >> sh16) & 0xFFFFu) | (((p1[3] >> sh16) & 0xFFFFu) << 16);
             }
-            // dt of both heads, de-interleaved: [entry][e][token]
-            const uint32_t lo01 = (raw[0] & 0xFFFFu) | (raw[1] << 16), lo23 = (raw[2] & 0xFFFFu) | (raw[3] << 16);
-            const uint32_t hi01 = (raw[0] >> 16) | (raw[1] & 0xFFFF0000u), hi23 = (raw[2] >> 16) | (raw[3] & 0xFFFF0000u);
+            const float a2 = __fmul_rn(__ldg(prm.A + h0i + e), kLog2e);
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float dv = (i & 1) ? bf16_hi(hv[i >> 1]) : bf16_lo(hv[i >> 1]);
+                v[i] = i == 0 ? __fmul_rn(dv, a2) : __fmaf_rn(dv, a2, v[i - 1]);
+            }
+            float incl = v[7];
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) {
+                const float q = __shfl_up_sync(0xffffffffu, incl, o, 16);
+                if (g >= o) incl = __fadd_rn(incl, q);
+            }
+            const float excl = __fsub_rn(incl, v[7]);
+            float mx = incl, mn = incl;
+#pragma unroll
+            for (int i = 0; i < 7; ++i) {
+                const float ac = __fadd_rn(excl, v[i]);
+                mx = fmaxf(mx, ac);
+                mn = fminf(mn, ac);
+            }
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) {
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o, 16));
+                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o, 16));
+            }
+            const int nv = nvalid - 8 * g;
+            bool dt_ok = true;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float dv = (i & 1) ? bf16_hi(hv[i >> 1]) : bf16_lo(hv[i >> 1]);
+                dt_ok = dt_ok && (nv <= i || fabsf(dv) >= 0x1p-40f);
+            }
+            // (mx - mn <= 128 is false for NaN, which then takes the exact form)
+            const bool fact = __all_sync(0xffffffffu, dt_ok && (mx - mn <= 128.f));
+            // Head0 = {m, tot, off1, off2, off3, a2, Dh, 0}; off q = the cumsum through token 32 q - 1;
+            // lane 16 e + f (f < 8) holds field f of head e
+            const float tot = __shfl_sync(0xffffffffu, incl, 15, 16), off1 = __shfl_sync(0xffffffffu, incl, 3, 16),
+                        off2 = __shfl_sync(0xffffffffu, incl, 7, 16), off3 = __shfl_sync(0xffffffffu, incl, 11, 16);
+            float hd_lane = 0.f;
+            if (g == 0) hd_lane = __fmul_rn(0.5f, __fadd_rn(mx, mn));
+            if (g == 1) hd_lane = tot;
+            if (g == 2) hd_lane = off1;
+            if (g == 3) hd_lane = off2;
+            if (g == 4) hd_lane = off3;
+            if (g == 5) hd_lane = a2;
+            if (g == 6 && prm.D) hd_lane = __ldg(prm.D + h0i + e);
             if (u + 1 < ntask) fetch(u + 1);  // the next pair task's dt, in flight while this one is written
             const int nsub = fact ? 1 : 2;
             for (int sub = 0; sub < nsub; ++sub) {
@@ -425,13 +442,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int d = td & (kRing - 1);
                 const int mode = fact ? kModePair : (sub == 0 ? kModeSingle0 : kModeSingle1);
                 const int flags = mode | ((sub == nsub - 1) ? (cu.w & kFlagLast) : 0);
-                asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(smem_u32(dts + (d * 2 + 0) * kQ + 4 * lane)),
-                             "r"(lo01), "r"(lo23)
-                             : "memory");
-                asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(smem_u32(dts + (d * 2 + 1) * kQ + 4 * lane)),
-                             "r"(hi01), "r"(hi23)
-                             : "memory");
-                if (lane < 16) reinterpret_cast<float *>(hds + 2 * d)[lane] = hd_lane;
+                *reinterpret_cast<uint4 *>(dts + (d * 2 + e) * kQ + 8 * g) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                if (g < 8) reinterpret_cast<float *>(hds + 2 * d)[8 * e + g] = hd_lane;
                 if (lane == 0) crd[d] = make_int4(cu.x, cu.y, cu.z, flags);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&dfull[d]);
@@ -592,6 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_ss(tmem + kTmY, cd0 + off, sd0 + 128 * kk, kIdY, kk > 0);
                     }
                     mma_commit(soff);
+                    mma_commit(&empty_cb[k]);  // C's last reader: the stage is free once this and dS are done
                     if (!wait_phase(&gp[j], (uint32_t)(t >> 1) & 1u, abort_flag, status)) break;
                     if (!wait_phase(&xpr[k], (uint32_t)(t >> 1) & 1u, abort_flag, status)) break;
                     tc_fence_after();
@@ -612,6 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_ss(tmem + kTmY + 64 * e, cd0 + off, sd0 + 128 * kk, kIdY1, kk > 0);
                     }
                     mma_commit(soff);
+                    mma_commit(&empty_cb[k]);
                     const uint64_t xd0 = sdesc(smem_u32(xslot(k) + e * kPanel), kPanel, 1024);
 #pragma unroll 1
                     for (int kk = 0; kk < kQ / 16; ++kk)
@@ -619,7 +633,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 mma_commit(&ydd[j]);
                 mma_commit(yfull);
-                mma_commit(&empty_cb[k]);
             }
             mma_commit(fin);
         }
@@ -1064,4 +1077,3 @@ cudaError_t tc_pair_fwd(const FwdProblem &p, void *ws, cudaStream_t s) {
 }
 
 }  // namespace ssd
-
