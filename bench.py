@@ -37,8 +37,14 @@ def peaks():
     return 6650.0, 1590.0, "fallback"
 
 
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ssd_fwd_tc_mamba2_2p7b_traffic.json")
-TC_SOURCE = os.path.join(ROOT, "state_space_sequence_chunked_b200", "csrc", "ssd_tc.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "k_ssd_pair_mamba2_2p7b_traffic.json")
+TC_SOURCE = os.path.join(ROOT, "state_space_sequence_chunked_b200", "csrc", "ssd_tc_pair.cu")
+
+
+def tc_kernel(wl):
+    """The tensor-core forward kernel that serves this workload: the head-pair kernel where
+    dstate is 128 and the heads of a group pair up, the one-head kernel otherwise."""
+    return "k_ssd_pair" if wl.dstate == 128 and (wl.nheads // wl.ngroups) % 2 == 0 else "k_ssd_tc<%d>" % wl.dstate
 
 
 def measured_traffic(wl, path):
@@ -74,6 +80,20 @@ def algorithmic(wl):
     return nbytes, flops
 
 
+def fwd_config(wl, path, l2):
+    """The config object of a forward line (both arms carry the same keys)."""
+    return {"workload": wl.name, "batch": wl.batch, "seqlen": wl.seqlen, "nheads": wl.nheads,
+            "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk,
+            "dt": wl.dt_dist, "path": path, "per_rank_batch": wl.batch, "l2": l2}
+
+
+def l2_note(wl):
+    e = 2 if wl.dtype == "bf16" else 4
+    mb = wl.batch * wl.seqlen * wl.nheads * wl.headdim * e / 1e6
+    return (f"inputs larger than L2 (x and y {mb:.1f} MB each per step vs 126 MB L2); no flush" if mb > 126
+            else f"x and y {mb:.1f} MB each per step: L2 flushed between steps")
+
+
 class ClockSampler:
     """SM clock and clock-event (throttle) reasons of this rank's GPU, read through NVML
     (the library nvidia-smi reports from) every 2 ms on a host thread; only samples
@@ -102,22 +122,37 @@ class ClockSampler:
         except Exception as e:  # no NVML on this host: the line says so
             self.error = f"{type(e).__name__}: {e}"
 
-    def _run(self):
+    def sample(self) -> bool:
         nv, h = self.nv, self.handle
+        t = time.perf_counter()
+        try:
+            sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+            rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+        except Exception as e:
+            self.error = f"{type(e).__name__}: {e}"
+            return False
+        self.samples.append((t, sm, rs))
+        return True
+
+    def _run(self):
         while not self.stop_ev.is_set():
-            t = time.perf_counter()
-            try:
-                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                self.samples.append((t, sm, rs))
-            except Exception as e:
-                self.error = f"{type(e).__name__}: {e}"
+            if not self.sample():
                 return
             time.sleep(0.002)
 
     def start(self):
         if self.thread is not None:
             self.thread.start()
+
+    def poll_until(self, event):
+        """Sample from the calling thread until `event` (recorded after the timed launches)
+        completes, so that even a timed region of a few milliseconds holds samples taken
+        while its kernels run."""
+        if self.handle is None:
+            return
+        while not event.query():
+            if not self.sample():
+                return
 
     def mark_start(self):
         self.t0 = time.perf_counter()
@@ -251,8 +286,8 @@ def reference_arm(args, wl):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * wl.batch * wl.seqlen / value, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "batch": wl.batch, "seqlen": wl.seqlen, "nheads": wl.nheads,
-                   "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk},
+        "config": fwd_config(wl, "oracle: fp64 recurrence on the host cores",
+                             "n/a (host memory; the oracle streams the inputs from RAM)"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": f"fp64 recurrence on {n} of {wl.batch * wl.nheads} (batch, head) streams "
                                    f"over all {wl.seqlen} tokens per step, extrapolated to the whole batch"},
@@ -303,6 +338,7 @@ def verify_main(args, wl):
     for _ in range(args.steps):
         step()
     ev1.record(stream)
+    clocks.poll_until(ev1)
     torch.cuda.synchronize()
     clocks.mark_end()
     barrier(ws)
@@ -418,6 +454,7 @@ def bwd_main(args, wl):
     for _ in range(args.steps):
         call(g)
     ev1.record(stream)
+    clocks.poll_until(ev1)
     torch.cuda.synchronize()
     clocks.mark_end()
     barrier(ws)
@@ -744,16 +781,32 @@ def main():
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(ws)
     torch.cuda.synchronize()
+    # inputs smaller than L2: each step timed on its own, with a write of 256 MB between steps
+    flush = None if wl.batch * wl.seqlen * wl.nheads * wl.headdim * (2 if wl.dtype == "bf16" else 4) > 126e6 \
+        else torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     clocks.mark_start()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
-    torch.cuda.synchronize()
+    if flush is None:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        clocks.poll_until(ev1)
+        torch.cuda.synchronize()
+        total_ms = ev0.elapsed_time(ev1)
+    else:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            step()
+            b.record(stream)
+        clocks.poll_until(evs[-1][1])
+        torch.cuda.synchronize()
+        total_ms = sum(a.elapsed_time(b) for a, b in evs)
     clocks.mark_end()
     barrier(ws)
     clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1) / args.steps
+    ms = total_ms / args.steps
     ms_max = reduce_max(ms, ws)
 
     tokens = wl.batch * wl.seqlen
@@ -812,13 +865,10 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
-            "config": {"workload": wl.name, "batch": wl.batch, "seqlen": wl.seqlen, "nheads": wl.nheads,
-                       "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk,
-                       "path": plan["path"], "per_rank_batch": wl.batch,
-                       "l2": "inputs larger than L2 (x and y 335.5 MB each per step vs 126 MB L2); no flush"},
+            "config": fwd_config(wl, plan["path"], l2_note(wl)),
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                          "frac": achieved / peak, "traffic": measured_traffic(wl, plan["path"]),
-                         "kernel": ("k_ssd_tc<%d> (the whole call: one launch after a status-word memset)" % wl.dstate
+                         "kernel": ("%s (the whole call: one launch after a status-word memset)" % tc_kernel(wl)
                                     if plan["path"] == "tcgen05" else
                                     "whole ssd_fwd call (%d launches)" % plan["kernels"]),
                          "peak_source": src, "alg_bytes": nbytes, "alg_flops": flops,

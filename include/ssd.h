@@ -108,11 +108,35 @@ ssd_status_t ssd_fwd_workspace_bytes(const ssd_shape_t *shape, ssd_dtype_t dtype
  *   h_final  [B, H, P, N]   fp32 or NULL   state after the last token
  *   workspace, workspace_bytes             >= ssd_fwd_workspace_bytes(...)
  * seqlen == 0 writes only h_final (= h0 or zeros); batch == 0 does nothing.
+ * The return value reports argument and launch errors only; the call is asynchronous.
+ * On SSD_PATH_TCGEN05 (ssd_fwd_plan) the kernel's CTAs wait on one another through
+ * bounded waits; if one runs out, the kernel abandons the call (y and h_final are then
+ * incomplete) and sets bit 0 of the workspace's first int32, the status word, which the
+ * call clears before launching. ssd_fwd_status reads it.
  */
 ssd_status_t ssd_fwd(const ssd_shape_t *shape, ssd_dtype_t dtype, const void *x, const void *dt,
                      const float *A, const void *Bm, const void *Cm, const float *D,
                      const float *h0, int64_t chunk, void *y, float *h_final, void *workspace,
                      size_t workspace_bytes, void *stream);
+
+/*
+ * Outcome of the last ssd_fwd on this workspace: synchronizes `stream`, then returns
+ * SSD_ERR_TIMEOUT if a bounded wait ran out (status word bit 0), SSD_ERR_CUDA if the
+ * kernel refused to run (any other bit: its shared memory was misaligned) or the
+ * stream reported an error, SSD_OK otherwise. Paths other than SSD_PATH_TCGEN05 have
+ * no waits and always give SSD_OK. shape, dtype and chunk are those of the call.
+ */
+ssd_status_t ssd_fwd_status(const ssd_shape_t *shape, ssd_dtype_t dtype, int64_t chunk,
+                            const void *workspace, void *stream);
+
+/*
+ * Test hook: the limit, in microseconds, of every bounded device-side wait in the
+ * kernels launched after this call, process-wide (0 restores the built-in 2 s).
+ * A small limit makes a wait between CTAs run out on purpose, so that the abort path
+ * (status word, drained copies, freed tensor memory) can be checked without a fault.
+ * Errors: SSD_ERR_INVALID_ARG outside 0..2000000.
+ */
+ssd_status_t ssd_set_wait_limit_us(int32_t us);
 
 /*
  * ssd_fwd for callers that cannot allocate device memory. No counterpart in
@@ -292,8 +316,10 @@ ssd_status_t ssd_cp_correct(const ssd_shape_t *shape, ssd_dtype_t dtype, const v
  *   dD        [H]            fp32 or NULL   out (also when D is NULL: the gradient at D = 0)
  *   dh0       [B, H, P, N]   fp32 or NULL   out (also when h0 is NULL: the gradient at h0 = 0)
  *   workspace, workspace_bytes              >= ssd_bwd_workspace_bytes(...)
- * Arithmetic is fp32 on CUDA cores for both dtypes. dBm and dCm are summed with fp32
- * atomics, so their last bits can differ between runs. batch == 0 zeroes dA and dD;
+ * Arithmetic follows ssd_bwd_plan: on SSD_PATH_MMA every product runs on tensor cores
+ * (mma.sync, bf16 operands, fp32 accumulation) and the rest in fp32; on SSD_PATH_SIMT
+ * everything is fp32 on CUDA cores. dBm and dCm are summed with fp32 atomics, so their
+ * last bits can differ between runs. batch == 0 zeroes dA and dD;
  * seqlen == 0 also writes dh0 = dh_final (or zeros).
  * Errors as ssd_fwd; SSD_ERR_UNSUPPORTED when headdim and dstate are too large for the
  * kernels' shared-memory tiles together (never for headdim, dstate <= 256).

@@ -43,6 +43,9 @@ _SIGS = {
     "ssd_fwd_workspace_bytes": ([ctypes.POINTER(ShapeT), ctypes.c_int, _i64, ctypes.POINTER(_sz)], ctypes.c_int),
     "ssd_fwd_plan": ([ctypes.POINTER(ShapeT), ctypes.c_int, _i64, ctypes.POINTER(PlanT)], ctypes.c_int),
     "ssd_fwd": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 7 + [_i64, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "ssd_fwd_static_scratch": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 7 + [_i64, _vp, _vp, _vp], ctypes.c_int),
+    "ssd_fwd_status": ([ctypes.POINTER(ShapeT), ctypes.c_int, _i64, _vp, _vp], ctypes.c_int),
+    "ssd_set_wait_limit_us": ([ctypes.c_int32], ctypes.c_int),
     "ssd_verify": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 7 + [_i64, _vp, _vp, _vp], ctypes.c_int),
     "ssd_select_state": ([ctypes.POINTER(ShapeT), _i64] + [_vp] * 5, ctypes.c_int),
     "ssd_advance_state": ([ctypes.POINTER(ShapeT), ctypes.c_int] + [_vp] * 5 + [_i64, _vp, _vp, _vp], ctypes.c_int),
@@ -141,8 +144,11 @@ def fwd_plan(batch, seqlen, nheads, headdim, ngroups, dstate, dtype_code, chunk)
 
 
 def ssd_fwd(x, dt, A, B, C, D=None, h0=None, *, chunk: int, y=None, h_final=None,
-            return_final_state: bool = True, workspace=None, stream=None):
-    """y, h_final = ssd_fwd(x [B,L,H,P], dt [B,L,H], A [H] f32, B/C [B,L,G,N], D [H] f32?, h0 [B,H,P,N] f32?)."""
+            return_final_state: bool = True, workspace=None, stream=None, check: bool = False):
+    """y, h_final = ssd_fwd(x [B,L,H,P], dt [B,L,H], A [H] f32, B/C [B,L,G,N], D [H] f32?, h0 [B,H,P,N] f32?).
+
+    check=True synchronizes the stream after the launch and raises SSDError (SSD_ERR_TIMEOUT)
+    if a bounded device-side wait ran out, which leaves y and h_final incomplete."""
     dev = _dev(x, dt, A, B, C, D, h0, y, h_final, workspace)
     Bsz, L, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
@@ -160,7 +166,24 @@ def ssd_fwd(x, dt, A, B, C, D=None, h0=None, *, chunk: int, y=None, h_final=None
                        _ptr(h0), chunk, _ptr(y), _ptr(h_final), _ptr(workspace), ws_bytes,
                        _stream(dev, stream))
     _check(st, "ssd_fwd")
+    if check:
+        _check(lib().ssd_fwd_status(ctypes.byref(shape), code, chunk, _ptr(workspace), _stream(dev, stream)),
+               "ssd_fwd")
     return y, h_final
+
+
+def fwd_status(shape_args, dtype_code, chunk, workspace, stream=None) -> int:
+    """Raw ssd_fwd_status code for the last ssd_fwd on `workspace` (synchronizes the stream).
+
+    shape_args = (batch, seqlen, nheads, headdim, ngroups, dstate)."""
+    shape = ShapeT(*shape_args)
+    dev = workspace.device if workspace is not None else torch.device("cuda", torch.cuda.current_device())
+    return lib().ssd_fwd_status(ctypes.byref(shape), dtype_code, chunk, _ptr(workspace), _stream(dev, stream))
+
+
+def set_wait_limit_us(us: int):
+    """Test hook: limit of every bounded device-side wait in later launches (0: the built-in 2 s)."""
+    _check(lib().ssd_set_wait_limit_us(int(us)), "ssd_set_wait_limit_us")
 
 
 def ssd_verify(h0, x, dt, A, B, C, D=None, *, states_out=None, y=None, return_states: bool = True,

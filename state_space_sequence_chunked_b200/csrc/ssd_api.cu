@@ -1,52 +1,19 @@
 // The C ABI: argument validation, workspace sizing and path selection.
 // Every check runs before any launch; on an error nothing is launched.
+#include <atomic>
+
 #include "ssd_internal.cuh"
 
 #define SSD_API extern "C" __attribute__((visibility("default")))
 
 namespace ssd {
+
+static std::atomic<int> g_wait_limit_us{0};
+int wait_limit_us() { return g_wait_limit_us.load(std::memory_order_relaxed); }
+
 namespace {
 
-constexpr int64_t kMaxDim = 256;      // headdim, dstate
-constexpr int64_t kMaxChunk = 256;
-constexpr int64_t kMaxGridYZ = 65535; // batch and nheads map to grid y/z
 constexpr int64_t kMaxVerifyK = 64;
-
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-ssd_status_t check_shape(const ssd_shape_t *s) {
-    if (!s) return SSD_ERR_INVALID_ARG;
-    if (s->batch < 0 || s->seqlen < 0 || s->nheads < 1 || s->headdim < 1 || s->ngroups < 1 ||
-        s->dstate < 1)
-        return SSD_ERR_INVALID_ARG;
-    if (s->nheads % s->ngroups != 0) return SSD_ERR_INVALID_ARG;
-    if (s->headdim > kMaxDim || s->dstate > kMaxDim) return SSD_ERR_UNSUPPORTED;
-    if (s->batch > kMaxGridYZ || s->nheads > kMaxGridYZ) return SSD_ERR_UNSUPPORTED;
-    return SSD_OK;
-}
-
-ssd_status_t check_dtype(ssd_dtype_t d) {
-    return (d == SSD_F32 || d == SSD_BF16) ? SSD_OK : SSD_ERR_INVALID_ARG;
-}
-
-ssd_status_t make_fwd(const ssd_shape_t *s, ssd_dtype_t dtype, int64_t chunk, FwdProblem *p) {
-    ssd_status_t st = check_shape(s);
-    if (st != SSD_OK) return st;
-    if ((st = check_dtype(dtype)) != SSD_OK) return st;
-    if (chunk < 1) return SSD_ERR_INVALID_ARG;
-    if (chunk > kMaxChunk) return SSD_ERR_UNSUPPORTED;
-    *p = FwdProblem{};
-    p->B = s->batch;
-    p->L = s->seqlen;
-    p->H = s->nheads;
-    p->P = s->headdim;
-    p->G = s->ngroups;
-    p->N = s->dstate;
-    p->Q = chunk;
-    p->nc = (s->seqlen + chunk - 1) / chunk;
-    p->dtype = dtype;
-    return SSD_OK;
-}
 
 ssd_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
 
@@ -141,6 +108,27 @@ SSD_API ssd_status_t ssd_fwd(const ssd_shape_t *shape, ssd_dtype_t dtype, const 
     p.y = y;
     p.h_final = h_final;
     return from_cuda(plan.path == SSD_PATH_TCGEN05 ? tc_fwd(p, workspace, s) : simt_fwd(p, workspace, s));
+}
+
+SSD_API ssd_status_t ssd_fwd_status(const ssd_shape_t *shape, ssd_dtype_t dtype, int64_t chunk,
+                                    const void *workspace, void *stream) {
+    FwdProblem p;
+    ssd_status_t st = make_fwd(shape, dtype, chunk, &p);
+    if (st != SSD_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SSD_ERR_CUDA;
+    if (plan_of(p).path != SSD_PATH_TCGEN05) return SSD_OK;  // the other paths have no waits
+    if (!workspace) return SSD_ERR_INVALID_ARG;
+    int32_t word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return SSD_ERR_CUDA;
+    if (word & 1) return SSD_ERR_TIMEOUT;
+    return word ? SSD_ERR_CUDA : SSD_OK;
+}
+
+SSD_API ssd_status_t ssd_set_wait_limit_us(int32_t us) {
+    if (us < 0 || us > 2000000) return SSD_ERR_INVALID_ARG;
+    g_wait_limit_us.store(us, std::memory_order_relaxed);
+    return SSD_OK;
 }
 
 SSD_API ssd_status_t ssd_verify(const ssd_shape_t *shape, ssd_dtype_t dtype, const float *h0,

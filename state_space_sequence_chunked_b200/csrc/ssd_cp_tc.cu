@@ -36,6 +36,7 @@ struct Params {
     int *status;
     long long L;
     int H, G, N, nblk, pairs_per_group, blocks_per_cta;
+    int wait_us;  // bounded-wait limit in microseconds (0: the built-in one)
 };
 
 // Shared memory (after 1024-byte alignment): S_in tile [N/64 panels], C tile [N/64 panels],
@@ -71,6 +72,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&ld_bar[1], 1);
         mbar_init(mma_bar, 1);
         *abort_flag = 0;
+        abort_flag[1] = prm.wait_us;  // bounded-wait limit (us; 0: the built-in one)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -250,6 +252,7 @@ cudaError_t cp_correct_tc_launch(const CpProblem &p, const void *dt, const float
     prm.bsum = bsum;
     prm.s_in = s_in;
     prm.status = status;
+    prm.wait_us = wait_limit_us();
     prm.L = p.L;
     prm.H = (int)p.H;
     prm.G = (int)p.G;

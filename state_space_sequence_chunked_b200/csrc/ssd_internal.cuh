@@ -46,6 +46,49 @@ struct CpProblem {
 constexpr size_t kWsAlign = 256;
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// ---- argument rules shared by every forward entry point ----------------------------
+constexpr int64_t kMaxDim = 256;       // headdim, dstate
+constexpr int64_t kMaxChunk = 256;
+constexpr int64_t kMaxGridYZ = 65535;  // batch and nheads map to grid y/z
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline ssd_status_t check_shape(const ssd_shape_t *s) {
+    if (!s) return SSD_ERR_INVALID_ARG;
+    if (s->batch < 0 || s->seqlen < 0 || s->nheads < 1 || s->headdim < 1 || s->ngroups < 1 || s->dstate < 1)
+        return SSD_ERR_INVALID_ARG;
+    if (s->nheads % s->ngroups != 0) return SSD_ERR_INVALID_ARG;
+    if (s->headdim > kMaxDim || s->dstate > kMaxDim) return SSD_ERR_UNSUPPORTED;
+    if (s->batch > kMaxGridYZ || s->nheads > kMaxGridYZ) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+inline ssd_status_t check_dtype(ssd_dtype_t d) { return (d == SSD_F32 || d == SSD_BF16) ? SSD_OK : SSD_ERR_INVALID_ARG; }
+
+// Shape, dtype and chunk checks, then the problem record (pointers unset).
+inline ssd_status_t make_fwd(const ssd_shape_t *s, ssd_dtype_t dtype, int64_t chunk, FwdProblem *p) {
+    ssd_status_t st = check_shape(s);
+    if (st != SSD_OK) return st;
+    if ((st = check_dtype(dtype)) != SSD_OK) return st;
+    if (chunk < 1) return SSD_ERR_INVALID_ARG;
+    if (chunk > kMaxChunk) return SSD_ERR_UNSUPPORTED;
+    *p = FwdProblem{};
+    p->B = s->batch;
+    p->L = s->seqlen;
+    p->H = s->nheads;
+    p->P = s->headdim;
+    p->G = s->ngroups;
+    p->N = s->dstate;
+    p->Q = chunk;
+    p->nc = (s->seqlen + chunk - 1) / chunk;
+    p->dtype = dtype;
+    return SSD_OK;
+}
+
+// Limit, in microseconds, of each bounded device-side wait of the next launches (0: the
+// built-in 2 s). Process-wide; set through ssd_set_wait_limit_us.
+int wait_limit_us();
+
 // ---- chunked path with fp32 CUDA-core arithmetic (exact path for fp32 inputs) ----
 size_t simt_fwd_workspace_bytes(const FwdProblem &p);
 cudaError_t simt_fwd(const FwdProblem &p, void *ws, cudaStream_t s);

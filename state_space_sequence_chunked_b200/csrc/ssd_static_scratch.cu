@@ -56,8 +56,6 @@ cudaError_t scratch_address(void **out) {
     return cudaSuccess;
 }
 
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 }  // namespace ssd
 
@@ -68,26 +66,10 @@ SSD_API ssd_status_t ssd_fwd_static_scratch(const ssd_shape_t *s, ssd_dtype_t dt
                                             const void *Cm, const float *D, const float *h0,
                                             int64_t chunk, void *y, float *h_final,
                                             void *stream) {
-    // Same argument rules as ssd_fwd.
-    if (!s) return SSD_ERR_INVALID_ARG;
-    if (s->batch < 0 || s->seqlen < 0 || s->nheads < 1 || s->headdim < 1 || s->ngroups < 1 ||
-        s->dstate < 1 || s->nheads % s->ngroups != 0)
-        return SSD_ERR_INVALID_ARG;
-    if (s->headdim > 256 || s->dstate > 256 || s->batch > 65535 || s->nheads > 65535)
-        return SSD_ERR_UNSUPPORTED;
-    if (dtype != SSD_F32 && dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
-    if (chunk < 1) return SSD_ERR_INVALID_ARG;
-    if (chunk > 256) return SSD_ERR_UNSUPPORTED;
-    FwdProblem p{};
-    p.B = s->batch;
-    p.L = s->seqlen;
-    p.H = s->nheads;
-    p.P = s->headdim;
-    p.G = s->ngroups;
-    p.N = s->dstate;
-    p.Q = chunk;
-    p.nc = (s->seqlen + chunk - 1) / chunk;
-    p.dtype = dtype;
+    // Same argument rules as ssd_fwd (one shared implementation).
+    FwdProblem p;
+    const ssd_status_t v = make_fwd(s, dtype, chunk, &p);
+    if (v != SSD_OK) return v;
     if (p.B == 0) return SSD_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (p.L == 0) {

@@ -104,6 +104,7 @@ struct Params {
     float *handover;     // [gridDim.x][P][N] state at the end of each CTA's first part
     long long L, total;  // total = B * H * nc tasks
     int H, G, nc;
+    int wait_us;         // bounded-wait limit in microseconds (0: the built-in one)
 };
 
 // The share of CTA i is [lo, hi) in (stream-major, block-minor) task order, run as
@@ -166,13 +167,13 @@ __device__ __forceinline__ void gprime_exact(uint32_t gaddr, int qtr, int row, f
 
 // Bounded spin on a hand-over counter in global memory.
 __device__ __noinline__ bool wait_flag(const int *flag, int want, volatile int *abort_flag, int *status) {
-    const unsigned long long t0 = now_ns();
+    const unsigned long long t0 = now_ns(), lim = wait_limit_ns(abort_flag);
     for (;;) {
         int v;
         asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
         if (v >= want) return true;
         if (*abort_flag) return false;
-        if (now_ns() - t0 > kWaitNs) {
+        if (now_ns() - t0 > lim) {
             *abort_flag = 1;
             atomicOr(status, 1);
             return false;
@@ -244,6 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(fin, 3);
         *abort_flag = 0;
+        abort_flag[1] = prm.wait_us;  // bounded-wait limit (us; 0: the built-in one)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kWarpG) {
@@ -756,6 +758,7 @@ cudaError_t launch(const FwdProblem &p, int *status, int *flags, float *handover
     prm.h_final = p.h_final;
     prm.y = static_cast<__nv_bfloat16 *>(p.y);
     prm.status = status;
+    prm.wait_us = wait_limit_us();
     prm.flags = flags;
     prm.handover = handover;
     prm.L = p.L;

@@ -97,6 +97,7 @@ struct Params {
     long long L;
     int total;           // B * (H / 2) * nc pair tasks
     int H, G, nc;
+    int wait_us;         // bounded-wait limit in microseconds (0: the built-in one)
 };
 
 // Share of CTA i in (pair stream, block) task order, run as [b0, hi), [a0, b0), [lo, a0): the
@@ -202,15 +203,29 @@ __device__ __forceinline__ void mul2(float w, uint32_t a, uint32_t b, uint32_t &
         : "r"(a), "r"(b), "f"(w));
 }
 
+// bf16 pair of w (y + d x) for fp32 y = (y0, y1) and a bf16 pair x, in packed fp32 pairs: the
+// same roundings as fmaf(d, x, y) then w * that, rounded to bf16.
+__device__ __forceinline__ uint32_t skip2_bf16(float w, float d, uint32_t y0, uint32_t y1, uint32_t x) {
+    uint32_t o;
+    asm("{\n\t.reg .b64 v, xx, ww, dd;\n\t.reg .b32 xl, xh;\n\t.reg .f32 lo, hi;\n\t"
+        "shl.b32 xl, %4, 16;\n\tand.b32 xh, %4, 0xFFFF0000;\n\t"
+        "mov.b64 v, {%2, %3};\n\tmov.b64 xx, {xl, xh};\n\tmov.b64 ww, {%1, %1};\n\tmov.b64 dd, {%5, %5};\n\t"
+        "fma.rn.f32x2 v, dd, xx, v;\n\tmul.rn.f32x2 v, v, ww;\n\t"
+        "mov.b64 {lo, hi}, v;\n\tcvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
+        : "=r"(o)
+        : "f"(w), "r"(y0), "r"(y1), "r"(x), "f"(d));
+    return o;
+}
+
 // Bounded spin on a hand-over counter in global memory.
 __device__ __noinline__ bool wait_flag(const int *flag, int want, volatile int *abort_flag, int *status) {
-    const unsigned long long t0 = now_ns();
+    const unsigned long long t0 = now_ns(), lim = wait_limit_ns(abort_flag);
     for (;;) {
         int v;
         asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
         if (v >= want) return true;
         if (*abort_flag) return false;
-        if (now_ns() - t0 > kWaitNs) {
+        if (now_ns() - t0 > lim) {
             *abort_flag = 1;
             atomicOr(status, 1);
             return false;
@@ -314,6 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&dsx[1], 1);
         mbar_init(soff, 1);
         *abort_flag = 0;
+        abort_flag[1] = prm.wait_us;  // bounded-wait limit (us; 0: the built-in one)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kWarpMma) {
@@ -667,11 +683,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint32_t r[32];
                         tmem_ld32(gaddr + 32 * jb, r);
                         tmem_wait_ld(r);
+                        if (jb < qtr) {  // wholly below the diagonal
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float v0 = 32 * jb + 2 * i <= row ? __uint_as_float(r[2 * i]) : 0.f;
-                            const float v1 = 32 * jb + 2 * i + 1 <= row ? __uint_as_float(r[2 * i + 1]) : 0.f;
-                            out[i] = pack_bf16(v0, v1);
+                            for (int i = 0; i < 16; ++i) out[i] = pack_bf16(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                        } else {  // the diagonal block: s = 32 jb + 2 i (+1) against row = 32 jb + lane
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const float v0 = 2 * i <= lane ? __uint_as_float(r[2 * i]) : 0.f;
+                                const float v1 = 2 * i + 1 <= lane ? __uint_as_float(r[2 * i + 1]) : 0.f;
+                                out[i] = pack_bf16(v0, v1);
+                            }
                         }
                     }
                     tmem_st16(gaddr + 16 * jb, out);
@@ -955,22 +976,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
 #pragma unroll
                     for (int c2 = 0; c2 < 2; ++c2) {
-                        float v[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(yv[8 * c2 + i]);
+                        const uint32_t *yy = yv + 8 * c2;
+                        uint4 o;
                         if (dd != 0.f) {
-                            v[0] = fmaf(dd, bf16_lo(xv[c2].x), v[0]);
-                            v[1] = fmaf(dd, bf16_hi(xv[c2].x), v[1]);
-                            v[2] = fmaf(dd, bf16_lo(xv[c2].y), v[2]);
-                            v[3] = fmaf(dd, bf16_hi(xv[c2].y), v[3]);
-                            v[4] = fmaf(dd, bf16_lo(xv[c2].z), v[4]);
-                            v[5] = fmaf(dd, bf16_hi(xv[c2].z), v[5]);
-                            v[6] = fmaf(dd, bf16_lo(xv[c2].w), v[6]);
-                            v[7] = fmaf(dd, bf16_hi(xv[c2].w), v[7]);
+                            o.x = skip2_bf16(rd, dd, yy[0], yy[1], xv[c2].x);
+                            o.y = skip2_bf16(rd, dd, yy[2], yy[3], xv[c2].y);
+                            o.z = skip2_bf16(rd, dd, yy[4], yy[5], xv[c2].z);
+                            o.w = skip2_bf16(rd, dd, yy[6], yy[7], xv[c2].w);
+                        } else {
+                            o = make_uint4(scale2_bf16(rd, __uint_as_float(yy[0]), __uint_as_float(yy[1])),
+                                           scale2_bf16(rd, __uint_as_float(yy[2]), __uint_as_float(yy[3])),
+                                           scale2_bf16(rd, __uint_as_float(yy[4]), __uint_as_float(yy[5])),
+                                           scale2_bf16(rd, __uint_as_float(yy[6]), __uint_as_float(yy[7])));
                         }
-                        *reinterpret_cast<uint4 *>(xs + swz(row, 2 * qq + c2)) =
-                            make_uint4(scale2_bf16(rd, v[0], v[1]), scale2_bf16(rd, v[2], v[3]),
-                                       scale2_bf16(rd, v[4], v[5]), scale2_bf16(rd, v[6], v[7]));
+                        *reinterpret_cast<uint4 *>(xs + swz(row, 2 * qq + c2)) = o;
                     }
                 }
                 fence_proxy_async();
@@ -1052,6 +1071,7 @@ cudaError_t tc_pair_fwd(const FwdProblem &p, void *ws, cudaStream_t s) {
     prm.h0 = p.h0;
     prm.h_final = p.h_final;
     prm.status = status;
+    prm.wait_us = wait_limit_us();
     prm.flags = flags;
     prm.handover = handover;
     prm.L = p.L;

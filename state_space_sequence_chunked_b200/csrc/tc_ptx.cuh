@@ -67,16 +67,23 @@ __device__ __forceinline__ unsigned long long now_ns() {
     return t;
 }
 
+// The limit of one bounded wait. abort_flag points at two shared words: [0] the CTA's abort
+// flag, [1] the launch's limit in microseconds (0: kWaitNs), set when the CTA starts.
+__device__ __forceinline__ unsigned long long wait_limit_ns(const volatile int *abort_flag) {
+    const int us = abort_flag[1];
+    return us > 0 ? (unsigned long long)us * 1000ull : kWaitNs;
+}
+
 // Bounded wait on a barrier phase. Returns false (and raises the abort flag and the
-// status word) when the phase does not complete within kWaitNs or another thread of
+// status word) when the phase does not complete within the limit or another thread of
 // the CTA has already aborted.
 static __device__ __noinline__ bool wait_phase_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                              int *status) {
-    const unsigned long long t0 = now_ns();
+    const unsigned long long t0 = now_ns(), lim = wait_limit_ns(abort_flag);
     for (;;) {
         if (mbar_try_sleep(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (now_ns() - t0 > kWaitNs) {
+        if (now_ns() - t0 > lim) {
             *abort_flag = 1;
             atomicOr(status, 1);
             return false;

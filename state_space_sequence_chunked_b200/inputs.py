@@ -7,7 +7,9 @@ binding) and the fp64 oracle can consume what it returns.
 Distributions (the SSD problem statement: input-dependent B, C and step size,
 a scalar decay rate per head, a per-head skip weight D):
     x   ~ N(0, 1)                       [B, L, H, P]
-    dt  = exp(U(ln 1e-3, ln 1e-1))      [B, L, H]
+    dt  = exp(U(ln 1e-3, ln 1e-1))      [B, L, H]     ("loguniform", the default), or
+    dt  = softplus(N(0, 1) + b_h),      [B, L, H]     ("softplus": a projection output plus a
+          b_h ~ U(-7, -2.3) per head                   per-head bias, as a Mamba-2 layer forms it)
     A_h = -exp(U(ln 1, ln 16))          [H]           (always fp32)
     B,C ~ N(0, 1) / sqrt(N)             [B, L, G, N]
     D   ~ N(0, 1)                       [H]           (always fp32)
@@ -39,20 +41,25 @@ class Workload:
     h0_std: float
     seed: int
     verify: bool = False
+    dt_dist: str = "loguniform"  # or "softplus" (see the module docstring)
 
     @property
     def tokens(self) -> int:
         return self.batch * self.seqlen
 
 
-# The five workloads: a tiny fp32 case, a 130M-like layer, the 2.7B-like layer
-# (the headline shape), a long-context large-state case and a spec-decode verify.
+# The workloads: a tiny fp32 case, a 130M-like layer, the 2.7B-like layer (the headline
+# shape), a long-context large-state case, a spec-decode verify, and the headline shape
+# with softplus-distributed step sizes.
 WORKLOADS = {
     "tiny_fp32": Workload("tiny_fp32", 1, 256, 4, 16, 16, 1, 64, "f32", 0.0, 0),
     "mamba2_130m": Workload("mamba2_130m", 8, 2048, 24, 64, 128, 1, 256, "bf16", 0.0, 1),
     "mamba2_2p7b": Workload("mamba2_2p7b", 4, 8192, 80, 64, 128, 1, 256, "bf16", 0.0, 2),
     "long_n256": Workload("long_n256", 1, 65536, 80, 64, 256, 1, 256, "bf16", 0.1, 3),
     "verify_k8": Workload("verify_k8", 64, 8, 32, 128, 128, 8, 8, "bf16", 0.1, 4, verify=True),
+    # the headline shape with step sizes spread as a trained layer's are (long tail to dt ~ 1+)
+    "mamba2_2p7b_softplus_dt": Workload("mamba2_2p7b_softplus_dt", 4, 8192, 80, 64, 128, 1, 256, "bf16", 0.0, 5,
+                                        dt_dist="softplus"),
 }
 
 
@@ -123,7 +130,11 @@ def draw(wl: Workload, *, batch=None, seqlen=None, seed=None, h0_std=None, zero_
     std = wl.h0_std if h0_std is None else h0_std
     rng = np.random.default_rng(wl.seed if seed is None else seed)
     x = rng.standard_normal((Bsz, L, H, P))
-    dt = np.exp(rng.uniform(math.log(1e-3), math.log(1e-1), size=(Bsz, L, H)))
+    if wl.dt_dist == "softplus":
+        v = rng.standard_normal((Bsz, L, H)) + rng.uniform(-7.0, -2.3, size=(H,))
+        dt = np.logaddexp(0.0, v)  # softplus, overflow-free
+    else:
+        dt = np.exp(rng.uniform(math.log(1e-3), math.log(1e-1), size=(Bsz, L, H)))
     A = -np.exp(rng.uniform(0.0, math.log(16.0), size=(H,)))
     Bm = rng.standard_normal((Bsz, L, G, N)) / math.sqrt(N)
     Cm = rng.standard_normal((Bsz, L, G, N)) / math.sqrt(N)

@@ -112,6 +112,42 @@ def test_fwd_rejects_before_launch(lib):
     assert fwd_call((0, 100, 4, 16, 1, 16), {k: None for k in GOOD}) == 0
 
 
+def static_call(shape, ptrs, chunk=64, dtype=B.SSD_BF16):
+    s = B.ShapeT(*shape)
+    p = {k: ctypes.c_void_p(v) if v else None for k, v in ptrs.items()}
+    return B.lib().ssd_fwd_static_scratch(ctypes.byref(s), dtype, p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"],
+                                          p["h0"], chunk, p["y"], p["hf"], None)
+
+
+def test_static_scratch_rejects_like_fwd(lib):
+    """The allocation-free entry point applies ssd_fwd's argument rules, before any launch."""
+    shape = (2, 100, 4, 16, 2, 16)
+    assert lib.ssd_fwd_static_scratch(None, 1, *([None] * 7), 64, None, None, None) == 1
+    for k in ("x", "dt", "A", "B", "C", "y"):
+        assert static_call(shape, {**GOOD, k: None}) == 1, k
+    for k in ("x", "dt", "A", "B", "C", "D", "y", "hf"):
+        assert static_call(shape, {**GOOD, k: GOOD[k] + 4}) == 3, k
+    assert static_call((2, 100, 4, 16, 3, 16), GOOD) == 1
+    assert static_call((-1, 100, 4, 16, 1, 16), GOOD) == 1
+    assert static_call((2, 100, 4, 300, 1, 16), GOOD) == 2
+    assert static_call((70000, 100, 4, 16, 1, 16), GOOD) == 2
+    assert static_call(shape, GOOD, chunk=0) == 1
+    assert static_call(shape, GOOD, chunk=257) == 2
+    assert static_call(shape, GOOD, dtype=3) == 1
+    assert static_call((0, 100, 4, 16, 1, 16), {k: None for k in GOOD}) == 0
+    # intermediates larger than the built-in array are refused (SSD_ERR_WORKSPACE)
+    assert static_call((64, 65536, 80, 64, 1, 128), GOOD, chunk=256) == 4
+
+
+def test_status_and_wait_limit_args(lib):
+    assert lib.ssd_set_wait_limit_us(-1) == 1
+    assert lib.ssd_set_wait_limit_us(2000001) == 1
+    assert lib.ssd_set_wait_limit_us(0) == 0
+    assert lib.ssd_fwd_status(None, 1, 64, None, None) == 1
+    assert lib.ssd_fwd_status(ctypes.byref(B.ShapeT(1, 10, 4, 16, 3, 16)), 1, 64, None, None) == 1
+    assert lib.ssd_fwd_status(ctypes.byref(B.ShapeT(1, 10, 4, 16, 1, 16)), 1, 0, None, None) == 1
+
+
 BWD_GOOD = dict(x=0x10000, dt=0x20000, A=0x30000, B=0x40000, C=0x50000, D=0x60000, h0=None, dy=0x70000,
                 dhf=None, dx=0x80000, ddt=0x90000, dA=0xa0000, dB=0xb0000, dC=0xc0000, dD=0xd0000, dh0=None,
                 ws=0xe0000)

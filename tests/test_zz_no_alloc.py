@@ -1,9 +1,11 @@
 """ssd_fwd_static_scratch: the forward pass for callers that cannot allocate
 device memory (a server that reserves all of HBM itself, a real-time loop, a
 plugin whose host owns every allocation). Its intermediates live in a built-in
-device array instead of a caller-provided workspace. Two calls in a row, on
-different inputs, must each match ssd_fwd (the entry point with a workspace) on
-the same inputs; a problem too large for the array must be refused.
+device array instead of a caller-provided workspace. Two calls in a row -- a
+larger problem, then a smaller one over the scratch the first left behind -- must
+each match the fp64 oracle and ssd_fwd (the entry point with a workspace) on the
+same inputs, without allocating device memory; a problem too large for the array
+must be refused.
 
 This file is collected last on purpose: it is the newest entry point, and a run
 that stops at the first failure has already run every other test by then."""
@@ -13,6 +15,7 @@ import dataclasses
 import pytest
 import torch
 
+import oracle
 from ssd_cases import TOL, rel_err, to_np
 from state_space_sequence_chunked_b200 import _binding as ssd
 from state_space_sequence_chunked_b200 import inputs
@@ -41,24 +44,49 @@ def call_static(g, h0, chunk, y, hf):
                         p(g["D"]), p(h0), chunk, p(y), p(hf), stream)
 
 
-def draw_case(dtype, seed, h0_std):
-    wl = dataclasses.replace(inputs.WORKLOADS["mamba2_130m"], batch=2, seqlen=700, nheads=6, ngroups=2,
+def draw_case(dtype, seed, h0_std, batch, seqlen, nheads):
+    wl = dataclasses.replace(inputs.WORKLOADS["mamba2_130m"], batch=batch, seqlen=seqlen, nheads=nheads, ngroups=2,
                              dtype=dtype, seed=seed, h0_std=h0_std)
     return wl, inputs.draw(wl)
 
 
+def device_bytes_in_use():
+    free, total = torch.cuda.mem_get_info()
+    return total - free
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_two_calls_match_ssd_fwd(cuda_device, dtype):
-    for call, (seed, std) in enumerate([(501, 0.1), (502, 0.0)]):
-        wl, d = draw_case(dtype, seed, std)
+def test_two_calls_match_oracle_and_ssd_fwd(cuda_device, dtype):
+    # the first call fills more of the scratch (more chunks and heads) than the second reads
+    cases = [(501, 0.1, 2, 1500, 8), (502, 0.0, 1, 700, 6)]
+    # one call first, so that loading the module (its code and the built-in array) is not
+    # counted as an allocation of the calls below
+    wl, d = draw_case(dtype, 500, 0.0, 1, 300, 2)
+    g = {k: d[k].torch(cuda_device) for k in ("x", "dt", "A", "B", "C", "D")}
+    assert call_static(g, None, 256, torch.empty_like(g["x"]), None) == 0
+    torch.cuda.synchronize()
+    for call, (seed, std, Bsz, L, H) in enumerate(cases):
+        wl, d = draw_case(dtype, seed, std, Bsz, L, H)
         g = {k: d[k].torch(cuda_device) for k in ("x", "dt", "A", "B", "C", "D")}
         h0 = d["h0"].torch(cuda_device) if d["h0"] is not None else None
-        need = ssd.fwd_plan(wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.ngroups, wl.dstate,
-                            ssd.SSD_BF16 if dtype == "bf16" else ssd.SSD_F32, 256)["workspace_bytes"]
+        # the static path runs the fp32 CUDA-core kernels whatever the dtype: size it by their plan
+        need = ssd.fwd_plan(wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.ngroups, wl.dstate, ssd.SSD_F32,
+                            256)["workspace_bytes"]
+        assert ssd.fwd_plan(wl.batch, wl.seqlen, wl.nheads, wl.headdim, wl.ngroups, wl.dstate, ssd.SSD_F32,
+                            256)["path"] == "simt"
         assert 0 < need <= SCRATCH_BYTES
         y = torch.full_like(g["x"], float("nan"))
         hf = torch.full((wl.batch, wl.nheads, wl.headdim, wl.dstate), float("nan"), device=cuda_device)
+        torch.cuda.synchronize()
+        alloc0, used0 = torch.cuda.memory_allocated(cuda_device), device_bytes_in_use()
         assert call_static(g, h0, 256, y, hf) == 0, f"call {call}"
+        torch.cuda.synchronize()
+        assert torch.cuda.memory_allocated(cuda_device) == alloc0, f"call {call}"
+        assert device_bytes_in_use() == used0, f"call {call}: device memory in use changed"
+        yr, hr = oracle.recurrent(d["x"].value, d["dt"].value, d["A"].value, d["B"].value, d["C"].value,
+                                  d["D"].value, d["h0"].value if d["h0"] is not None else None)
+        assert rel_err(to_np(y), yr) <= TOL[dtype], f"call {call}"
+        assert rel_err(to_np(hf), hr) <= TOL[dtype], f"call {call}"
         y_ref, hf_ref = ssd.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], h0, chunk=256)
         torch.cuda.synchronize()
         assert rel_err(to_np(y), to_np(y_ref)) <= TOL[dtype], f"call {call}"
