@@ -19,8 +19,11 @@
 // Between the two products one pass over the accumulator (E warps) recovers S_{t+1}, writes
 // its bf16 copy for step 4 of block t+1 and rescales the accumulator for block t+1.
 //
-// A block is factored for a head when its A_cs range is at most 128 (log2 units) and every
-// valid token has |dt| >= 2^-40. A pair task in which either head's block is not factored is
+// A block is factored for a head when its A_cs range is at most 192 (log2 units) and every
+// valid token has |dt| >= 2^-40. The row and column factors then stay within 2^+-96, which
+// leaves 2^31 of the exponent range that fp32 and bf16 share (up to 2^127) for |dt x| and the
+// 128-term sums of the products; a decay factor below 2^-126 flushes to 0, as the true value
+// is negligible next to the terms it is added to. A pair task in which either head's block is not factored is
 // run as two single-head tasks, each in the elementwise (exact) form for its head e, with
 // N = 64 products on that head's columns only:
 //   x_e stays in its half of the x slot; X'_e[s] = exp(A_cs_e[127] - A_cs_e[s]) dt_s x_s goes
@@ -249,17 +252,21 @@ __device__ __forceinline__ uint32_t ld_dt_pair(const __nv_bfloat16 *p, uint64_t 
 // Per (task, head) factors of the state pass: gamma = exp(A_cs[127]), dsc = the chunk state's
 // factor (exp(A_cs[127] - m) factored, 1 exact), sg = the scale of the bf16 copy (exp(m)
 // factored, 1 exact); a head that is not in a single-head task keeps its state: all 1.
+// Per head and block: dsc scales the block's chunk-state product (the accumulator then holds
+// S_{t+1} / dsc), sg the bf16 copy of the state for the state-to-output product, rs the state
+// the accumulator holds before the product ((gamma / dsc) S, gamma = exp(A_cs[127])). In the
+// factored form sg = rs = exp(m) exactly; in the exact form of the head the state enters
+// unscaled (sg = 1) and the accumulator holds gamma S; the other head's state passes through.
 struct StateF {
-    float gam, dsc, sg;
+    float dsc, sg, rs;
 };
 __device__ __forceinline__ StateF state_factors(const Head0 &hd, int mode, int e) {
     StateF f{1.f, 1.f, 1.f};
     if (mode == kModePair) {
-        f.gam = ex2(hd.tot);
         f.dsc = ex2(hd.tot - hd.m);
-        f.sg = ex2(hd.m);
+        f.sg = f.rs = ex2(hd.m);
     } else if (mode == kModeSingle0 + e) {
-        f.gam = ex2(hd.tot);
+        f.rs = ex2(hd.tot);
     }
     return f;
 }
@@ -438,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 dt_ok = dt_ok && (nv <= i || fabsf(dv) >= 0x1p-40f);
             }
             // (mx - mn <= 128 is false for NaN, which then takes the exact form)
-            const bool fact = __all_sync(0xffffffffu, dt_ok && (mx - mn <= 128.f));
+            const bool fact = __all_sync(0xffffffffu, dt_ok && (mx - mn <= 192.f));
             // Head0 = {m, tot, off1, off2, off3, a2, Dh, 0}; off q = the cumsum through token 32 q - 1;
             // lane 16 e + f (f < 8) holds field f of head e
             const float tot = __shfl_sync(0xffffffffu, incl, 15, 16), off1 = __shfl_sync(0xffffffffu, incl, 3, 16),
@@ -865,28 +872,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (starts && cd.z != 0 &&
                 !(ok = __all_sync(0xffffffffu, wait_flag(prm.flags + blockIdx.x - 1, 256, abort_flag, status))))
                 break;
-            const float rs = f.gam / f.dsc;
             if (!starts) {
-                // steady state: straight from the accumulator, with the two factors folded
-                const float c1 = f.sg * dsc_prev, c2 = rs * dsc_prev;
+                // steady state, straight from the accumulator: S_t = dsc_prev acc, then sg S_t and
+                // rs S_t. In the factored form sg = rs, and the two factors fold into one,
+                // cs = sg dsc_prev, unless that product is below the normal range (both factors
+                // can reach 2^-96); then they are applied one after the other.
+                const float cs = f.sg * dsc_prev;
+                const bool fold = f.sg == f.rs && cs >= 0x1p-120f;
+                const float c0 = fold ? cs : dsc_prev;
 #pragma unroll 1
                 for (int qq = 0; qq < 4; ++qq) {
                     uint32_t r[16], v[16];
                     tmem_ld16(sacc + 16 * qq, r);
                     tmem_wait_ld();
+#pragma unroll
+                    for (int p = 0; p < 16; p += 2) mul2(c0, r[p], r[p + 1], v[p], v[p + 1]);
                     uint4 o0, o1;
-                    o0.x = scale2_bf16(c1, __uint_as_float(r[0]), __uint_as_float(r[1]));
-                    o0.y = scale2_bf16(c1, __uint_as_float(r[2]), __uint_as_float(r[3]));
-                    o0.z = scale2_bf16(c1, __uint_as_float(r[4]), __uint_as_float(r[5]));
-                    o0.w = scale2_bf16(c1, __uint_as_float(r[6]), __uint_as_float(r[7]));
-                    o1.x = scale2_bf16(c1, __uint_as_float(r[8]), __uint_as_float(r[9]));
-                    o1.y = scale2_bf16(c1, __uint_as_float(r[10]), __uint_as_float(r[11]));
-                    o1.z = scale2_bf16(c1, __uint_as_float(r[12]), __uint_as_float(r[13]));
-                    o1.w = scale2_bf16(c1, __uint_as_float(r[14]), __uint_as_float(r[15]));
+                    if (fold) {
+                        o0 = make_uint4(pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1])),
+                                        pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3])),
+                                        pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5])),
+                                        pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7])));
+                        o1 = make_uint4(pack_bf16(__uint_as_float(v[8]), __uint_as_float(v[9])),
+                                        pack_bf16(__uint_as_float(v[10]), __uint_as_float(v[11])),
+                                        pack_bf16(__uint_as_float(v[12]), __uint_as_float(v[13])),
+                                        pack_bf16(__uint_as_float(v[14]), __uint_as_float(v[15])));
+                    } else {  // v holds S_t
+                        o0 = make_uint4(scale2_bf16(f.sg, __uint_as_float(v[0]), __uint_as_float(v[1])),
+                                        scale2_bf16(f.sg, __uint_as_float(v[2]), __uint_as_float(v[3])),
+                                        scale2_bf16(f.sg, __uint_as_float(v[4]), __uint_as_float(v[5])),
+                                        scale2_bf16(f.sg, __uint_as_float(v[6]), __uint_as_float(v[7])));
+                        o1 = make_uint4(scale2_bf16(f.sg, __uint_as_float(v[8]), __uint_as_float(v[9])),
+                                        scale2_bf16(f.sg, __uint_as_float(v[10]), __uint_as_float(v[11])),
+                                        scale2_bf16(f.sg, __uint_as_float(v[12]), __uint_as_float(v[13])),
+                                        scale2_bf16(f.sg, __uint_as_float(v[14]), __uint_as_float(v[15])));
+#pragma unroll
+                        for (int p = 0; p < 16; p += 2) mul2(f.rs, v[p], v[p + 1], v[p], v[p + 1]);
+                    }
                     *reinterpret_cast<uint4 *>(pb + swz(row, 2 * qq)) = o0;
                     *reinterpret_cast<uint4 *>(pb + swz(row, 2 * qq + 1)) = o1;
-#pragma unroll
-                    for (int p = 0; p < 16; p += 2) mul2(c2, r[p], r[p + 1], v[p], v[p + 1]);
                     tmem_st16(sacc + 16 * qq, v);
                 }
             } else {
@@ -915,7 +939,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     *reinterpret_cast<uint4 *>(pb + swz(row, 2 * qq + 1)) = o1;
                     uint32_t v[16];
 #pragma unroll
-                    for (int p = 0; p < 16; ++p) v[p] = __float_as_uint(rs * S[p]);
+                    for (int p = 0; p < 16; ++p) v[p] = __float_as_uint(f.rs * S[p]);
                     tmem_st16(sacc + 16 * qq, v);
                 }
                 if (ends) publish(cprev);

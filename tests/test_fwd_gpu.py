@@ -124,17 +124,21 @@ def test_tensor_core_products_in_isolation(cuda_device, what, nheads):
 @pytest.mark.parametrize("chunk", [128, 256])
 def test_wide_decay_and_zero_step_blocks(cuda_device, chunk):
     """The tensor-core path evaluates a block in factored form only when its decay range
-    is at most 2^128 and no token has |dt| < 2^-40; other blocks take the elementwise
-    form. Here the two kinds alternate within streams: head 0 has one block with dt = 1
-    (range 128 * 2 * log2 e = 369), head 1 has A = 0 (no decay), head 2 has one token with
-    dt = 0, and head 3 decays by 2^-11.5 per token everywhere."""
-    d = _tc_case(21, batch=2, seqlen=700, nheads=4, h0_std=0.2)
+    is small enough (2^128 for the one-head kernel, 2^192 for the head-pair kernel) and no
+    token has |dt| < 2^-40; other blocks take the elementwise form. Here the kinds alternate
+    within streams: head 0 has one block with dt = 1 (range 128 * 2 * log2 e = 369), head 1
+    has A = 0 (no decay), head 2 has one token with dt = 0, head 3 decays by 2^-11.5 per
+    token everywhere, head 4 has one block of range 128 * 0.9 * log2 e = 166 (factored by
+    the pair kernel, elementwise by the one-head kernel) and head 5 one of range 191."""
+    d = _tc_case(21, batch=2, seqlen=700, nheads=6, h0_std=0.2)
     dt = d["dt"].value.copy()
     dt[0, 128:256, 0] = 1.0
     dt[1, 300, 2] = 0.0
     dt[:, :, 3] = 0.5
+    dt[0, 256:384, 4] = 0.9
+    dt[1, 384:512, 5] = 1.0
     d["dt"] = inputs.Tensor(dt, "bf16")
-    d["A"] = inputs.Tensor(np.array([-2.0, 0.0, -4.0, -16.0]), "f32")
+    d["A"] = inputs.Tensor(np.array([-2.0, 0.0, -4.0, -16.0, -1.0, -1.035]), "f32")
     assert plan_of(d, chunk)["path"] == "tcgen05"
     check_full(d, chunk, cuda_device)
 
