@@ -143,6 +143,15 @@ __device__ __forceinline__ float quarter_cumsum(float dt, float a2, float off, i
 struct Head0 {
     float m, tot, off1, off2, off3, a2, Dh, pad;
     __device__ __forceinline__ float off(int q) const { return q == 0 ? 0.f : (q == 1 ? off1 : (q == 2 ? off2 : off3)); }
+    // the middle of quarter q's A_cs span (its bounds: the cumsum before it and at its end)
+    __device__ __forceinline__ float qmid(int q) const { return 0.5f * (off(q) + (q == 3 ? tot : off(q + 1))); }
+    // The exact form factors a block by quarters unless a quarter spans more than 224 of A_cs
+    // (its factors then stay within 2^+-112); past that it takes exp(A_cs[l] - A_cs[s]) element
+    // by element.
+    __device__ __forceinline__ bool fine() const {
+        const float w = fmaxf(fmaxf(-off1, off1 - off2), fmaxf(off2 - off3, off3 - tot));
+        return !(w <= 224.f);  // (NaN: element by element)
+    }
 };
 
 // w x for a bf16 pair x, rounded once to bf16 up to a few units in 2^-17: w is split into
@@ -269,6 +278,106 @@ __device__ __forceinline__ StateF state_factors(const Head0 &hd, int mode, int e
         f.rs = ex2(hd.tot);
     }
     return f;
+}
+
+// ---------------------------------------------------------------------------------------------
+// The exact form's two per-task jobs, out of line: they run only for blocks whose decay range
+// is too wide for the factored form, and kept inline they would lengthen the code every
+// factored block runs through.
+
+// T warp (rows 32 qtr .. 32 qtr + 31) for head ea of an exact task, once C B^T is in the G
+// buffer at gaddr (this warp's lanes): G' of head ea in place, then C's rows scaled by
+// exp(A_cs[l]) in place (the state term's row factor, which the exact form cannot share with the
+// G' product). Factored by quarters: with X'''_s = exp(mid_q(s) - A_cs[s]) dt_s x_s (mid_q the
+// middle of s's quarter), G'[l,s] = (C B^T)[l,s] exp(A_cs[l] - mid_q(s)), one factor per row and
+// quarter; a quarter spanning more than 224 of A_cs instead takes X'''_s = dt_s x_s and
+// G'[l,s] = (C B^T)[l,s] exp(A_cs[l] - A_cs[s]) element by element.
+__device__ __noinline__ void t_exact(unsigned char *cst, uint32_t gaddr, const Head0 hx, const __nv_bfloat16 *dtrow,
+                                     int qtr, int lane) {
+    const int row = (qtr << 5) | lane;
+    float acs_r;
+    if (!hx.fine()) {
+        acs_r = quarter_cumsum(__bfloat162float(dtrow[row]), hx.a2, hx.off(qtr), lane);
+#pragma unroll 1
+        for (int jb = 0; jb < 4; ++jb) {
+            uint32_t out[16];
+            if (jb > qtr) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) out[i] = 0u;
+            } else {
+                uint32_t r[32];
+                tmem_ld32(gaddr + 32 * jb, r);
+                const float rf = ex2(acs_r - hx.qmid(jb));
+                tmem_wait_ld(r);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    float v0 = __uint_as_float(r[2 * i]), v1 = __uint_as_float(r[2 * i + 1]);
+                    if (jb == qtr) {  // the diagonal quarter: s = 32 jb + 2 i (+1) against l = 32 jb + lane
+                        v0 = 2 * i <= lane ? v0 : 0.f;
+                        v1 = 2 * i + 1 <= lane ? v1 : 0.f;
+                    }
+                    out[i] = scale2_bf16(rf, v0, v1);
+                }
+            }
+            tmem_st16(gaddr + 16 * jb, out);
+        }
+    } else {
+        // the columns need step 0 of every quarter, so this warp runs all four
+        float acq[4];  // token 32 jb + lane
+#pragma unroll
+        for (int jb = 0; jb < 4; ++jb)
+            acq[jb] = quarter_cumsum(__bfloat162float(dtrow[32 * jb + lane]), hx.a2, hx.off(jb), lane);
+        acs_r = qtr == 0 ? acq[0] : (qtr == 1 ? acq[1] : (qtr == 2 ? acq[2] : acq[3]));
+#pragma unroll 1
+        for (int pc = 0; pc < 8; ++pc) {
+            const int jb = pc >> 1;
+            uint32_t out[8];
+            if (jb > qtr) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) out[i] = 0u;
+            } else {
+                const float aj = jb == 0 ? acq[0] : (jb == 1 ? acq[1] : (jb == 2 ? acq[2] : acq[3]));
+                uint32_t r[16];
+                tmem_ld16(gaddr + 16 * pc, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float v[2];
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int ci = 16 * (pc & 1) + 2 * i + hh, col = 32 * jb + ci;
+                        const float ac = __shfl_sync(0xffffffffu, aj, ci);
+                        v[hh] = col <= row ? __uint_as_float(r[2 * i + hh]) * ex2(acs_r - ac) : 0.f;
+                    }
+                    out[i] = pack_bf16(v[0], v[1]);
+                }
+            }
+            tmem_st8(gaddr + 8 * pc, out);
+        }
+    }
+    const float el = ex2(acs_r);
+    scale_row(cst, cst, row, el);
+    scale_row(cst + kPanel, cst + kPanel, row, el);
+    fence_proxy_async();
+}
+
+// X warp (row `row` of the block) of an exact task of head ea. xw (the warp belongs to head ea):
+// X'''_ea[row] (see t_exact) into the other head's half of the slot, x_ea staying in its own
+// for the chunk-state product and the skip term. Otherwise, once C B^T has read B: B[row,:] *=
+// exp(A_cs[127] - A_cs[row]) dt_row in place, the chunk-state product's decay.
+__device__ __noinline__ void x_exact(unsigned char *x_own, unsigned char *x_other, unsigned char *bst, const Head0 hd,
+                                     const __nv_bfloat16 *dtrow, int qtr, int lane, bool xw) {
+    const int row = (qtr << 5) | lane;
+    const float dt_r = __bfloat162float(dtrow[row]);
+    const float acs_r = quarter_cumsum(dt_r, hd.a2, hd.off(qtr), lane);
+    if (xw) {
+        scale_row(x_own, x_other, row, hd.fine() ? dt_r : ex2(hd.qmid(qtr) - acs_r) * dt_r);
+    } else {
+        const float w = ex2(hd.tot - acs_r) * dt_r;
+        scale_row(bst, bst, row, w);
+        scale_row(bst + kPanel, bst + kPanel, row, w);
+    }
+    fence_proxy_async();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -590,9 +699,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t xd0 = sdesc(smem_u32(xslot(k)), kPanel, 1024);
 #pragma unroll 1
                     for (int kk = 0; kk < kQ / 16; ++kk) mma_ss(tmem + kTmS, ad0 + 128 * kk, xd0 + 128 * kk, kIdDs, 1);
-                } else {  // head e's columns only, from X'_e in the other half
+                } else {  // head e's columns only: B' (rows of B scaled by the X warps) times raw x_e
                     const int e = mode == kModeSingle0 ? 0 : 1;
-                    const uint64_t xd0 = sdesc(smem_u32(xslot(k) + (1 - e) * kPanel), kPanel, 1024);
+                    const uint64_t xd0 = sdesc(smem_u32(xslot(k) + e * kPanel), kPanel, 1024);
 #pragma unroll 1
                     for (int kk = 0; kk < kQ / 16; ++kk)
                         mma_ss(tmem + kTmS + 64 * e, ad0 + 128 * kk, xd0 + 128 * kk, kIdDs1, 1);
@@ -649,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     mma_commit(soff);
                     mma_commit(&empty_cb[k]);
-                    const uint64_t xd0 = sdesc(smem_u32(xslot(k) + e * kPanel), kPanel, 1024);
+                    const uint64_t xd0 = sdesc(smem_u32(xslot(k) + (1 - e) * kPanel), kPanel, 1024);
 #pragma unroll 1
                     for (int kk = 0; kk < kQ / 16; ++kk)
                         mma_ts(tmem + kTmY + 64 * e, tmem + kTmG + 128 * j + 8 * kk, xd0 + 128 * kk, kIdY1, 1);
@@ -663,7 +772,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= kWarpT && warp < kWarpX) {
         // ------------------------------------------------------------- T: G' (and the exact form's C rows)
         const int qtr = warp & 3;
-        const int row = (qtr << 5) | lane;
         const uint32_t lane_off = (uint32_t)(qtr * 32) << 16;
         for (int t = 0;; ++t) {
             const int k = t & 1, j = t & 1;
@@ -705,56 +813,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st16(gaddr + 16 * jb, out);
                 }
             } else {
-                // exact form for head e. The G' columns need step 0 of every quarter, so this warp
-                // runs all four.
-                const int e = mode == kModeSingle0 ? 0 : 1;
-                const Head0 hd = hds[2 * dq + e];
-                const float De = hd.Dh, a2 = hd.a2;
-                float acq[4], dtq[4];  // token 32 jb + lane
-#pragma unroll
-                for (int jb = 0; jb < 4; ++jb) {
-                    dtq[jb] = __bfloat162float(dts[(dq * 2 + e) * kQ + 32 * jb + lane]);
-                    acq[jb] = quarter_cumsum(dtq[jb], a2, hd.off(jb), lane);
-                }
-                const float acs_r = qtr == 0 ? acq[0] : (qtr == 1 ? acq[1] : (qtr == 2 ? acq[2] : acq[3]));
-                // G'_e[l,s] = G[l,s] exp(A_cs[l] - A_cs[s]) dt_s for s < l, G[l,l] dt_l + D_e, 0 above
-#pragma unroll 1
-                for (int pc = 0; pc < 8; ++pc) {
-                    const int jb = pc >> 1;
-                    uint32_t out[8];
-                    if (jb > qtr) {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) out[i] = 0u;
-                    } else {
-                        const float aj = jb == 0 ? acq[0] : (jb == 1 ? acq[1] : (jb == 2 ? acq[2] : acq[3]));
-                        const float dj = jb == 0 ? dtq[0] : (jb == 1 ? dtq[1] : (jb == 2 ? dtq[2] : dtq[3]));
-                        uint32_t r[16];
-                        tmem_ld16(gaddr + 16 * pc, r);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            float v[2];
-#pragma unroll
-                            for (int hh = 0; hh < 2; ++hh) {
-                                const int ci = 16 * (pc & 1) + 2 * i + hh, col = 32 * jb + ci;
-                                const float ac = __shfl_sync(0xffffffffu, aj, ci);
-                                const float dc = __shfl_sync(0xffffffffu, dj, ci);
-                                const float gv = __uint_as_float(r[2 * i + hh]);
-                                v[hh] = col < row ? gv * ex2(acs_r - ac) * dc : (col == row ? fmaf(gv, dc, De) : 0.f);
-                            }
-                            out[i] = pack_bf16(v[0], v[1]);
-                        }
-                    }
-                    tmem_st8(gaddr + 8 * pc, out);
-                }
-                // C[row,:] *= exp(A_cs[row]) in place (C B^T is done with C): the state term's row
-                // factor, which the exact form cannot share with the G' product
-                if (!wait_warp(&full_cb[k], (uint32_t)(t >> 1) & 1u, abort_flag, status)) break;
-                const float el = ex2(acs_r);
-                unsigned char *cs = cb_c(k);
-                scale_row(cs, cs, row, el);
-                scale_row(cs + kPanel, cs + kPanel, row, el);
-                fence_proxy_async();
+                const int ea = mode == kModeSingle0 ? 0 : 1;
+                t_exact(cb_c(k), gaddr, hds[2 * dq + ea], dts + (dq * 2 + ea) * kQ, qtr, lane);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -771,18 +831,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int4 cd = crd[dq];
             if (cd.w & kFlagEnd) break;
             const int mode = cd.w & 3;
-            const bool act = mode == kModePair || mode == kModeSingle0 + e;
-            if (!wait_warp(&full_x[k], (uint32_t)(t >> 1) & 1u, abort_flag, status)) break;
-            if (act) {
+            if (mode == kModePair) {
+                if (!wait_warp(&full_x[k], (uint32_t)(t >> 1) & 1u, abort_flag, status)) break;
                 const Head0 hd = hds[2 * dq + e];
                 unsigned char *xs = xslot(k) + e * kPanel;
                 const float dt_r = __bfloat162float(dts[(dq * 2 + e) * kQ + row]);
                 const float acs_r = quarter_cumsum(dt_r, hd.a2, hd.off(qtr), lane);
-                if (mode == kModePair)
-                    scale_row(xs, xs, row, ex2(hd.m - acs_r) * dt_r);
-                else
-                    scale_row(xs, xslot(k) + (1 - e) * kPanel, row, ex2(hd.tot - acs_r) * dt_r);
+                scale_row(xs, xs, row, ex2(hd.m - acs_r) * dt_r);
                 fence_proxy_async();
+            } else {  // exact form of head ea: X''' (its warps) or B's rows (the other head's)
+                const int ea = mode == kModeSingle0 ? 0 : 1;
+                if (!wait_warp(ea == e ? &full_x[k] : &gfull[k], (uint32_t)(t >> 1) & 1u, abort_flag, status)) break;
+                tc_fence_after();
+                x_exact(xslot(k) + ea * kPanel, xslot(k) + (1 - ea) * kPanel, cb_b(k), hds[2 * dq + ea],
+                        dts + (dq * 2 + ea) * kQ, qtr, lane, ea == e);
             }
             mbar_arrive(&xpr[k]);
         }
@@ -835,7 +897,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         float dsc_prev = 1.f;
         int4 cprev = make_int4(0, 0, 0, 0);
         for (int t = 0; ok; ++t) {
-            const int k = t & 1;
             const int dq = t & (kRing - 1);
             if (!(ok = wait_warp(&dfull[dq], (uint32_t)(t >> 2) & 1u, abort_flag, status))) break;
             const int4 cd = crd[dq];
@@ -974,6 +1035,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float acs_r = quarter_cumsum(dt_r, hd.a2, hd.off(qtr), lane);
                 rd = ex2(acs_r - hd.m);
                 dd = dt_r != 0.f ? hd.Dh / dt_r : 0.f;
+            } else if (act) {
+                dd = hds[2 * dq + e].Dh;  // exact form: y = Y + D x, x still in this head's half
             }
             if (!wait_warp(yfull, (uint32_t)t & 1u, abort_flag, status)) break;
             tc_fence_after();
