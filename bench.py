@@ -52,7 +52,9 @@ def measured_traffic(wl, path):
     capture, if that capture was taken of the kernel source as it is now; else None."""
     import hashlib
 
-    if wl.name != "mamba2_2p7b" or path != "tcgen05" or not os.path.exists(TRAFFIC_FILE):
+    from state_space_sequence_chunked_b200 import inputs
+
+    if wl != inputs.WORKLOADS["mamba2_2p7b"] or path != "tcgen05" or not os.path.exists(TRAFFIC_FILE):
         return None
     rec = json.load(open(TRAFFIC_FILE))
     src = hashlib.sha256(open(TC_SOURCE, "rb").read()).hexdigest()
@@ -723,6 +725,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba2_2p7b")
+    ap.add_argument("--seqlen", type=int, default=None,
+                    help="override the workload's sequence length (a smaller case for profiler captures)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--block", action="store_true",
@@ -740,6 +744,10 @@ def main():
     from state_space_sequence_chunked_b200 import inputs
 
     wl = inputs.WORKLOADS[args.workload]
+    if args.seqlen is not None:
+        import dataclasses
+
+        wl = dataclasses.replace(wl, seqlen=args.seqlen)
     if args.bwd:
         if args.impl == "reference" or wl.verify:
             raise SystemExit("--bwd times this library's backward of a forward workload")
