@@ -43,6 +43,8 @@
 // own TMA loads and MMAs, frees TMEM and returns.
 #include <algorithm>
 
+// the E threads keep a 64-value state row live across their waits
+#define SSD_INLINE_SLOW_WAIT
 #include "tc_ptx.cuh"
 
 namespace ssd {
@@ -50,7 +52,6 @@ namespace tc {
 
 constexpr int kQ = 128;  // tokens per diagonal block
 constexpr int kP = 64;   // head dimension handled by this path
-constexpr int kThreads = 384;
 constexpr int kWarpTma = 0, kWarpG = 1, kWarpDs = 2, kWarpYs = 3, kWarpE = 8;  // warps 4-7: T
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -59,6 +60,10 @@ struct Cfg {
     // N = 128: double-buffered input stages and S^T. N = 256: one of each (the wider B, C and
     // S^T fill shared memory).
     static constexpr bool kWide = N == 256;
+    // E warps: one set of four per 128 state rows (each thread keeps one state row of 64
+    // values in registers); the first set also runs the epilogue
+    static constexpr int kESets = N / 128;
+    static constexpr int kThreads = 32 * (kWarpE + 4 * kESets);
     static constexpr int kStages = kWide ? 1 : 2;
     static constexpr int kYBufs = 2;
     static constexpr int kStBufs = kWide ? 1 : 2;
@@ -136,21 +141,22 @@ __device__ __forceinline__ Share share_of(long long total, int nc, int i, int G)
 // time; volatile, so that they stay after the barrier wait that makes those values valid.
 __device__ __forceinline__ void gprime_exact(uint32_t gaddr, int qtr, int row, float acs_r, const float *acsW,
                                           const float *dk, float Dh) {
+    // 16 columns per TMEM load (the 512-thread N = 256 configuration caps a thread at 128 registers)
 #pragma unroll 1
-    for (int jb = 0; jb < 4; ++jb) {
-        uint32_t out[16];
-        if (jb > qtr) {
+    for (int pc = 0; pc < 8; ++pc) {
+        uint32_t out[8];
+        if ((pc >> 1) > qtr) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) out[i] = 0u;
+            for (int i = 0; i < 8; ++i) out[i] = 0u;
         } else {
-            uint32_t r[32];
-            tmem_ld32(gaddr + 32 * jb, r);
-            tmem_wait_ld(r);
-            const uint32_t aw = (uint32_t)__cvta_generic_to_shared(acsW + 32 * jb);
-            const uint32_t dw = (uint32_t)__cvta_generic_to_shared(dk + 32 * jb);
+            uint32_t r[16];
+            tmem_ld16(gaddr + 16 * pc, r);
+            tmem_wait_ld();
+            const uint32_t aw = (uint32_t)__cvta_generic_to_shared(acsW + 16 * pc);
+            const uint32_t dw = (uint32_t)__cvta_generic_to_shared(dk + 16 * pc);
 #pragma unroll  // whole: r and out stay in registers
-            for (int i = 0; i < 16; ++i) {
-                const int s = 32 * jb + 2 * i;
+            for (int i = 0; i < 8; ++i) {
+                const int s = 16 * pc + 2 * i;
                 float a0, a1, d0, d1;
                 asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(a0), "=f"(a1) : "r"(aw + 8 * i));
                 asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(d0), "=f"(d1) : "r"(dw + 8 * i));
@@ -161,7 +167,7 @@ __device__ __forceinline__ void gprime_exact(uint32_t gaddr, int qtr, int row, f
                 out[i] = pack_bf16(v0, v1);
             }
         }
-        tmem_st16(gaddr + 16 * jb, out);
+        tmem_st8(gaddr + 8 * pc, out);
     }
 }
 
@@ -183,7 +189,7 @@ __device__ __noinline__ bool wait_flag(const int *flag, int want, volatile int *
 }
 
 template <int N>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<N>::kThreads, 1)
     k_ssd_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
              const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y, const Params prm) {
     using Cf = Cfg<N>;
@@ -226,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&full_bc[i], 1);
             mbar_init(&full_x[i], 1);
             mbar_init(&empty_bc[i], 3);
-            mbar_init(&empty_x[i], 4 + 4 + 2);
+            mbar_init(&empty_x[i], 4 + 4 * Cf::kESets + 2);
             mbar_init(&xpr[i], 128);
         }
         for (int i = 0; i < 2; ++i) {
@@ -236,9 +242,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < DB; ++i) {
             mbar_init(&dsdone[i], 1);
-            mbar_init(&dsfree[i], 128);
+            mbar_init(&dsfree[i], 128 * Cf::kESets);
         }
-        for (int i = 0; i < SB; ++i) mbar_init(&sready[i], 128);
+        for (int i = 0; i < SB; ++i) mbar_init(&sready[i], 128 * Cf::kESets);
         for (int i = 0; i < YB; ++i) {
             mbar_init(&yfull[i], 1);
             mbar_init(&yfree[i], 128);
@@ -568,11 +574,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------- E: state chain + epilogue
-        const int qtr = warp & 3;
+        const int qtr = warp & 3, set = Cf::kESets == 1 ? 0 : (warp - kWarpE) >> 2;
         const int row = (qtr << 5) | lane;
         const uint32_t lane_off = (uint32_t)(qtr * 32) << 16;
-        constexpr int NH = N / 128;  // state rows per thread: n = row + 128 i
-        float Sr[NH][kP];
+        const int nrow = row + 128 * set;  // this thread's state row n
+        float Sr[kP];
         // S_in^T of task t, bf16, scaled by s = exp(m) of task t in the factored form (1 in the
         // exact form), into its buffer
         auto write_st = [&](int t) -> bool {
@@ -584,17 +590,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) bulk_wait_read();
             __syncwarp();
 #pragma unroll
-            for (int i = 0; i < NH; ++i) {
-                const int n = row + 128 * i;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint4 o;
-                    o.x = scale2_bf16(sg, Sr[i][8 * ch + 0], Sr[i][8 * ch + 1]);
-                    o.y = scale2_bf16(sg, Sr[i][8 * ch + 2], Sr[i][8 * ch + 3]);
-                    o.z = scale2_bf16(sg, Sr[i][8 * ch + 4], Sr[i][8 * ch + 5]);
-                    o.w = scale2_bf16(sg, Sr[i][8 * ch + 6], Sr[i][8 * ch + 7]);
-                    *reinterpret_cast<uint4 *>(stb + swz(n, ch)) = o;
-                }
+            for (int ch = 0; ch < 8; ++ch) {
+                uint4 o;
+                o.x = scale2_bf16(sg, Sr[8 * ch + 0], Sr[8 * ch + 1]);
+                o.y = scale2_bf16(sg, Sr[8 * ch + 2], Sr[8 * ch + 3]);
+                o.z = scale2_bf16(sg, Sr[8 * ch + 4], Sr[8 * ch + 5]);
+                o.w = scale2_bf16(sg, Sr[8 * ch + 6], Sr[8 * ch + 7]);
+                *reinterpret_cast<uint4 *>(stb + swz(nrow, ch)) = o;
             }
             fence_proxy_async();
             mbar_arrive(&sready[t % SB]);
@@ -608,18 +610,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c == 0) {
                 const long long base = (long long)sidx * kP * N;
 #pragma unroll
-                for (int i = 0; i < NH; ++i)
-#pragma unroll
-                    for (int p = 0; p < kP; ++p)
-                        Sr[i][p] = prm.h0 ? prm.h0[base + (long long)p * N + row + 128 * i] : 0.f;
+                for (int p = 0; p < kP; ++p) Sr[p] = prm.h0 ? prm.h0[base + (long long)p * N + nrow] : 0.f;
                 return true;
             }
-            if (!wait_flag(prm.flags + blockIdx.x - 1, 128, abort_flag, status)) return false;
+            // every E thread of the previous CTA has written its row and counted itself
+            if (!wait_flag(prm.flags + blockIdx.x - 1, 128 * Cf::kESets, abort_flag, status)) return false;
             const float *src = prm.handover + (long long)(blockIdx.x - 1) * kP * N;
 #pragma unroll
-            for (int i = 0; i < NH; ++i)
-#pragma unroll
-                for (int p = 0; p < kP; ++p) Sr[i][p] = __ldcg(src + p * N + row + 128 * i);
+            for (int p = 0; p < kP; ++p) Sr[p] = __ldcg(src + p * N + nrow);
             return true;
         };
         // End of a piece: the final state of the stream, or the hand-over to the next CTA.
@@ -630,16 +628,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (prm.h_final) {
                     const long long base = (long long)sidx * kP * N;
 #pragma unroll
-                    for (int i = 0; i < NH; ++i)
-#pragma unroll
-                        for (int p = 0; p < kP; ++p) prm.h_final[base + (long long)p * N + row + 128 * i] = Sr[i][p];
+                    for (int p = 0; p < kP; ++p) prm.h_final[base + (long long)p * N + nrow] = Sr[p];
                 }
             } else {
                 float *dst = prm.handover + (long long)blockIdx.x * kP * N;
 #pragma unroll
-                for (int i = 0; i < NH; ++i)
-#pragma unroll
-                    for (int p = 0; p < kP; ++p) __stcg(dst + p * N + row + 128 * i, Sr[i][p]);
+                for (int p = 0; p < kP; ++p) __stcg(dst + p * N + nrow, Sr[p]);
                 __threadfence();
                 atomicAdd(prm.flags + blockIdx.x, 1);
             }
@@ -660,16 +654,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             {
                 const float gam = ex2(blk.x), dsc = ex2(blk.x - blk.y);
 #pragma unroll
-                for (int i = 0; i < NH; ++i) {
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + ds_col(t) + 64 * set + 32 * half + lane_off, r);
+                    tmem_wait_ld(r);
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        uint32_t r[32];
-                        tmem_ld32(tmem + ds_col(t) + 64 * i + 32 * half + lane_off, r);
-                        tmem_wait_ld(r);
-#pragma unroll
-                        for (int q = 0; q < 32; q += 2)
-                            fma2_state(Sr[i][32 * half + q], Sr[i][32 * half + q + 1], gam, dsc, r[q], r[q + 1]);
-                    }
+                    for (int q = 0; q < 32; q += 2)
+                        fma2_state(Sr[32 * half + q], Sr[32 * half + q + 1], gam, dsc, r[q], r[q + 1]);
                 }
                 tc_fence_before();
                 mbar_arrive(&dsfree[db]);
@@ -686,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // inside Y)
             if (!(ok = wait_warp(&yfull[yb], (uint32_t)(t / YB) & 1u, abort_flag, status))) break;
             tc_fence_after();
-            {
+            if (set == 0) {
                 // y rows of this warp (32 tokens x 64 values) are staged, 128-byte swizzled, in its
                 // 4 KB slice of the S^T buffer of task t (free: Y_off of task t is done) and written
                 // by one bulk tensor store.
@@ -772,7 +763,7 @@ cudaError_t launch(const FwdProblem &p, int *status, int *flags, float *handover
     // over), which a cooperative launch guarantees.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(Cfg<N>::kThreads);
     cfg.dynamicSmemBytes = Cfg<N>::kSmemAlloc;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

@@ -74,7 +74,7 @@ constexpr int kOffDt = kOffS + 2 * kPanel;        // bf16 dt [ring][2 heads][128
 constexpr int kOffHd = kOffDt + kRing * 2 * kQ * 2;  // Head0 [ring][2 heads]: step-0 scalars
 constexpr int kOffCrd = kOffHd + kRing * 2 * 32;  // int4 [ring]: task descriptor
 constexpr int kOffBar = kOffCrd + kRing * 16;
-constexpr int kNumBars = 33;
+constexpr int kNumBars = 35;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;  // TMEM base, abort flag
 constexpr int kSmemBytes = kOffMisc + 16;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -189,11 +189,6 @@ __device__ __forceinline__ void scale_row(const unsigned char *src, unsigned cha
     }
 }
 
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), "r"(v[0]),
-                 "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-                 : "memory");
-}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
@@ -395,8 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *full_cb = bar;          // [2] C, B of the stage landed
     uint64_t *empty_cb = bar + 2;     // [2] C B^T, chunk-state and Y commits
     uint64_t *full_x = bar + 4;       // [2] x of the slot landed
-    uint64_t *empty_x = bar + 6;      // [2] y of the slot stored (8 O warps); also frees the
-                                      //     descriptor two tasks back
+    uint64_t *empty_x0 = bar + 6;     // [2] head 0's half of the slot free: its y stored (4 O warps)
+    uint64_t *empty_x1 = bar + 33;    // [2] the same for head 1's half
     uint64_t *xpr = bar + 8;          // [2] X'' (or X') written (X warps)
     uint64_t *gfull = bar + 10;       // [2] C B^T in G buffer j
     uint64_t *gp = bar + 12;          // [2] G' written (T)
@@ -429,7 +424,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&full_cb[i], 1);
             mbar_init(&empty_cb[i], 2);  // the two MMA issuers
             mbar_init(&full_x[i], 1);
-            mbar_init(&empty_x[i], 8);  // the 8 O warps
+            mbar_init(&empty_x0[i], 4);  // head 0's 4 O warps
+            mbar_init(&empty_x1[i], 4);  // head 1's
             mbar_init(&xpr[i], 256);  // the 8 X warps
             mbar_init(&gfull[i], 1);
             mbar_init(&gp[i], 128);
@@ -635,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_phase(&dfull[d], (uint32_t)(tx >> 2) & 1u, abort_flag, status)) break;
                 const int4 cd = crd[d];
                 if (cd.w & kFlagEnd) break;
-                if (tx >= 2 && !wait_phase(&empty_x[k], (uint32_t)((tx - 2) >> 1) & 1u, abort_flag, status)) break;
+                const uint32_t pe = (uint32_t)((tx - 2) >> 1) & 1u;  // slot k's previous use
                 const int d1 = (tx + 1) & (kRing - 1);
                 if (mbar_test(&dfull[d1], (uint32_t)((tx + 1) >> 2) & 1u)) {
                     const int4 cf = crd[d1];
@@ -647,12 +643,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 const int mode = cd.w & 3, h0i = 2 * cd.y, t0 = cd.z * kQ;
+                // each half as soon as its previous y is out (the exact form writes the other half too)
                 if (mode == kModePair) {
                     mbar_arrive_tx(&full_x[k], 2 * kTxXHead);
+                    if (tx >= 2 && !wait_phase(&empty_x0[k], pe, abort_flag, status)) break;
                     tma_load_4d_hint(xslot(k), &tm_x, &full_x[k], 0, h0i, t0, cd.x, pol_stream);
+                    last_x[k] = tx;  // (an abort here still drains this load, with the bounded wait)
+                    if (tx >= 2 && !wait_phase(&empty_x1[k], pe, abort_flag, status)) break;
                     tma_load_4d_hint(xslot(k) + kPanel, &tm_x, &full_x[k], 0, h0i + 1, t0, cd.x, pol_stream);
                 } else {
                     const int e = mode == kModeSingle0 ? 0 : 1;
+                    if (tx >= 2 && !(wait_phase(&empty_x0[k], pe, abort_flag, status) &&
+                                     wait_phase(&empty_x1[k], pe, abort_flag, status)))
+                        break;
                     mbar_arrive_tx(&full_x[k], kTxXHead);
                     tma_load_4d_hint(xslot(k) + e * kPanel, &tm_x, &full_x[k], 0, h0i + e, t0, cd.x, pol_stream);
                 }
@@ -1095,7 +1098,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&empty_x[k]);
+                mbar_arrive(e ? &empty_x1[k] : &empty_x0[k]);
                 mbar_arrive(&dfree[dq]);
             }
         }

@@ -77,8 +77,17 @@ __device__ __forceinline__ unsigned long long wait_limit_ns(const volatile int *
 // Bounded wait on a barrier phase. Returns false (and raises the abort flag and the
 // status word) when the phase does not complete within the limit or another thread of
 // the CTA has already aborted.
-static __device__ __noinline__ bool wait_phase_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                             int *status) {
+// Out of line by default (the call costs only the kernels whose waits are rarely slow); a
+// translation unit whose threads keep many registers live across waits defines
+// SSD_INLINE_SLOW_WAIT before including this header, as the call's register saves would go
+// to local memory there.
+#ifdef SSD_INLINE_SLOW_WAIT
+#define SSD_SLOW_WAIT_LINKAGE __forceinline__
+#else
+#define SSD_SLOW_WAIT_LINKAGE __noinline__
+#endif
+static __device__ SSD_SLOW_WAIT_LINKAGE bool wait_phase_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                                      int *status) {
     const unsigned long long t0 = now_ns(), lim = wait_limit_ns(abort_flag);
     for (;;) {
         if (mbar_try_sleep(bar, parity)) return true;
@@ -216,6 +225,11 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" : SSD_W8(0), SSD_W8(8), SSD_W8(16), SSD_W8(24)::"memory");
 }
 #undef SSD_W8
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), "r"(v[0]),
+                 "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
