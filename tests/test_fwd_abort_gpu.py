@@ -5,7 +5,8 @@ through which a CTA hands a cut stream's state to the next) gives up after a lim
 raises the CTA's abort flag and sets bit 0 of the status word at the start of the
 workspace. Here the limit is cut to 1 us through the library's test hook, on shapes
 with at least as many streams as SMs (so streams are cut between CTAs and states are
-handed over). The call must come back, report SSD_ERR_TIMEOUT through ssd_fwd_status,
+handed over), for both kernels: head pairs (an even head count at N = 128) and single
+heads (an odd head count, or N = 256). The call must come back, report SSD_ERR_TIMEOUT through ssd_fwd_status,
 and leave the GPU usable: the next call, with the normal limit, must match the oracle
 (it allocates the same tensor memory, which the aborted CTAs therefore released).
 No fault, trap or unbounded wait is involved."""
@@ -29,7 +30,7 @@ def _case(dstate, nheads, seed):
     return wl, inputs.draw(wl)
 
 
-@pytest.mark.parametrize("dstate,nheads", [(128, 320), (256, 160)])
+@pytest.mark.parametrize("dstate,nheads", [(128, 320), (256, 320), (128, 161), (256, 161)])
 def test_wait_limit_runs_out_then_next_call_is_exact(cuda_device, dstate, nheads):
     wl, d = _case(dstate, nheads, 900 + dstate)
     plan = plan_of(d, wl.chunk)

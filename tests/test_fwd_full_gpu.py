@@ -63,10 +63,11 @@ def test_every_stream_full_size(cuda_device, name):
     print(f"{name}: worst stream y {ey.max():.3e}, h_final {eh.max():.3e}")
 
 
-@pytest.mark.parametrize("dstate,nheads", [(128, 300), (256, 150)])
+@pytest.mark.parametrize("dstate,nheads", [(128, 300), (256, 300), (128, 151), (256, 153)])
 def test_cut_streams_every_stream(cuda_device, dstate, nheads):
-    """150 streams (head pairs for N = 128, heads for N = 256) of 16 blocks over 148 CTAs:
-    the shares are about 16.2 blocks long, so nearly every stream is split between two
+    """150 to 300 streams of 16 blocks over 148 CTAs: head pairs (300 heads at N = 128, the
+    head-pair kernel) or single heads (an odd head count, or N = 256: the one-head kernel).
+    The shares are 16.2 to 32.4 blocks long, so nearly every stream is split between two
     CTAs at a different block, and its state crosses through the hand-over buffer."""
     wl = dataclasses.replace(inputs.WORKLOADS["mamba2_2p7b"], batch=1, seqlen=2048, nheads=nheads, dstate=dstate,
                              h0_std=0.2, seed=40 + dstate)
