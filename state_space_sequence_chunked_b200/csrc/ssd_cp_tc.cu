@@ -7,14 +7,16 @@
 // Over one 128-token block and two heads of one group it is a single matrix product
 //     Y[t, (h, p)] = sum_n C[t, n] S_in[h, p, n]        (M = 128 tokens, N = 2 x 64, K = dstate)
 // followed by a per-(token, head) scaling. A CTA takes one head pair of one batch row and a run
-// of consecutive 128-token blocks, all of which share S_in:
-//   - the 256 threads write S_in once, converted to bf16, K-major with 128-byte swizzle;
-//   - per block, TMA brings C (same layout, 64-column panels) and the two heads' y tiles (two y
-//     buffers: the next block's tiles load while this block's are updated);
-//   - one thread issues dstate / 16 MMAs (M = 128, N = 128) into a TMEM accumulator;
-//   - warps 0-1 form the decay factors of the two heads;
-//   - each warp reads its TMEM lane quarter for one head and updates the y tile in shared
-//     memory, and one thread stores both tiles with TMA.
+// of consecutive 128-token blocks, all of which share S_in, and pipelines them:
+//   - the 8 epilogue warps first write S_in once, converted to bf16, K-major with 128-byte
+//     swizzle;
+//   - warp 8 (one thread) loads each block's C (one buffer: it is free once the block's MMAs
+//     are done) and the two heads' y tiles (two buffers), issues the block's dstate / 16 MMAs
+//     (M = 128, N = 128) into one of two TMEM accumulators, and stores each block's y tiles
+//     once the epilogue has updated them, so block i+1's loads and MMAs run during block i's
+//     epilogue;
+//   - in the epilogue, warps 0-1 form the decay factors of the two heads; each warp reads its
+//     TMEM lane quarter for one head and updates the y tile in shared memory.
 // Every wait is bounded; a wait that runs out sets bit 0 of *status (when given) and the CTA
 // skips the rest of its work.
 #include <algorithm>
@@ -28,7 +30,8 @@ using namespace tc;
 constexpr int kBlk = 128;      // tokens per CTA
 constexpr int kP = 64;         // head dimension this kernel takes
 constexpr int kPanel = 16384;  // one 64-column panel of a 128-row K-major tile, bytes
-constexpr int kThreads = 256;
+constexpr int kThreads = 288;  // 8 epilogue warps and the producer warp
+constexpr int kEpi = 256;      // epilogue threads
 
 struct Params {
     const __nv_bfloat16 *dt;
@@ -40,8 +43,9 @@ struct Params {
 };
 
 // Shared memory (after 1024-byte alignment): S_in tile [N/64 panels], C tile [N/64 panels],
-// y tiles [2 buffers][2 heads][128 rows x 128 B], cum [2][128] fp32, barriers, TMEM base, abort.
-__host__ __device__ constexpr int smem_bytes(int N) { return 2 * (N / 64) * kPanel + 4 * kPanel + 2 * kBlk * 4 + 64; }
+// y tiles [2 buffers][2 heads][128 rows x 128 B], cum [2 buffers][2 heads][128] fp32, 8 barriers,
+// TMEM base, abort flag and wait limit.
+__host__ __device__ constexpr int smem_bytes(int N) { return 2 * (N / 64) * kPanel + 4 * kPanel + 4 * kBlk * 4 + 128; }
 
 __global__ void __launch_bounds__(kThreads, 1)
     k_correct_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y, const Params prm) {
@@ -52,10 +56,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char *s_tile = sm;
     unsigned char *c_tile = sm + npan * kPanel;
     unsigned char *y_tile = sm + 2 * npan * kPanel;  // [2][2][16 KB]
-    float *cum = reinterpret_cast<float *>(y_tile + 4 * kPanel);
-    uint64_t *ld_bar = reinterpret_cast<uint64_t *>(cum + 2 * kBlk);  // [2]: C and y of block i, i % 2
-    uint64_t *mma_bar = ld_bar + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_bar + 1);
+    float *cum = reinterpret_cast<float *>(y_tile + 4 * kPanel);       // [2][2][128]
+    uint64_t *ld_bar = reinterpret_cast<uint64_t *>(cum + 4 * kBlk);  // [2] C and y tiles of block i landed (i % 2)
+    uint64_t *mma_bar = ld_bar + 2;    // [2] the MMAs of block i done (accumulator i % 2)
+    uint64_t *acc_free = ld_bar + 4;   // [2] accumulator i % 2 read out by the epilogue
+    uint64_t *y_done = ld_bar + 6;     // [2] y tiles of buffer i % 2 updated by the epilogue
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ld_bar + 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int local_status = 0;
     int *status = prm.status ? prm.status : &local_status;
@@ -68,16 +74,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long L = prm.L;
 
     if (tid == 0) {
-        mbar_init(&ld_bar[0], 1);
-        mbar_init(&ld_bar[1], 1);
-        mbar_init(mma_bar, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ld_bar[i], 1);
+            mbar_init(&mma_bar[i], 1);
+            mbar_init(&acc_free[i], kEpi);
+            mbar_init(&y_done[i], kEpi);
+        }
         *abort_flag = 0;
         abort_flag[1] = prm.wait_us;  // bounded-wait limit (us; 0: the built-in one)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(128)
+                     "r"(256)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -86,32 +95,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t load_bytes = (uint32_t)(npan * kPanel + 2 * kPanel);
-    // C panels and the two heads' y tiles of the CTA's block i, into y buffer i % 2
-    auto issue_loads = [&](int i) {
-        const int t0 = (blk0 + i) * kBlk;
-        uint64_t *bar = &ld_bar[i & 1];
-        mbar_arrive_tx(bar, load_bytes);
-        for (int pn = 0; pn < npan; ++pn) tma_load_4d(c_tile + pn * kPanel, &tm_c, bar, 64 * pn, g, t0, b);
-        for (int e = 0; e < 2; ++e) tma_load_4d(y_tile + ((i & 1) * 2 + e) * kPanel, &tm_y, bar, 0, h0 + e, t0, b);
-    };
-    if (tid == 0 && nb > 0) issue_loads(0);
-    // S_in of the two heads -> bf16, K-major: row r = 64 e + p, 16-byte chunk (n / 8) in panel n / 64.
-    // chunks = 128 N / 8 is a multiple of 4 * kThreads: four chunks' loads are issued per thread
-    // before any of them is converted.
-    {
+
+    if (warp < 8) {
+        // S_in of the two heads -> bf16, K-major: row r = 64 e + p, 16-byte chunk (n / 8) in panel
+        // n / 64. chunks = 128 N / 8 is a multiple of 4 * kEpi: four chunks' loads are issued per
+        // thread before any of them is converted.
         const float *src = prm.s_in + ((long long)b * prm.H + h0) * kP * N;  // the two heads are adjacent
         const int chunks = kBlk * (N / 8);
-        for (int i0 = tid; i0 < chunks; i0 += 4 * kThreads) {
+        for (int i0 = tid; i0 < chunks; i0 += 4 * kEpi) {
             float4 lo[4], hi[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int i = i0 + u * kThreads, r = i / (N / 8), cc = i % (N / 8);
+                const int i = i0 + u * kEpi, r = i / (N / 8), cc = i % (N / 8);
                 lo[u] = reinterpret_cast<const float4 *>(src + (long long)r * N)[2 * cc];
                 hi[u] = reinterpret_cast<const float4 *>(src + (long long)r * N)[2 * cc + 1];
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int i = i0 + u * kThreads, r = i / (N / 8), cc = i % (N / 8);
+                const int i = i0 + u * kEpi, r = i / (N / 8), cc = i % (N / 8);
                 uint4 o;
                 o.x = pack_bf16(lo[u].x, lo[u].y);
                 o.y = pack_bf16(lo[u].z, lo[u].w);
@@ -120,77 +121,121 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<uint4 *>(s_tile + (cc >> 3) * kPanel + swz(r, cc & 7)) = o;
             }
         }
+        fence_proxy_async();  // the generic-proxy writes of S_in are visible to the tensor cores
     }
-    fence_proxy_async();  // the generic-proxy writes of S_in are visible to the tensor cores
     __syncthreads();
 
-    const int q = warp & 3, e = warp >> 2, row = 32 * q + lane;  // epilogue: TMEM lane quarter, head
-    const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + 64 * e;
-    bool ok = true;
-    int last_mma = -1, last_ld = nb > 0 ? 0 : -1;  // thread 0: the latest block whose MMAs / loads it issued
-    for (int i = 0; i < nb && ok; ++i) {
-        const int blk = blk0 + i;
-        const long long t0 = (long long)blk * kBlk;
-        if (warp < 2) {  // decay factors exp(cumulative dt A) of head h0 + warp over the block's tokens
-            const int h = h0 + warp;
-            const float a = prm.A[h];
-            const float *bs = prm.bsum + ((long long)b * prm.H + h) * prm.nblk;
-            float pre = 0.f;
-            for (int k = lane; k < blk; k += 32) pre += bs[k];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) pre += __shfl_xor_sync(0xffffffffu, pre, o);
-            const long long tt = t0 + 4 * lane;
-            float v[4];
-#pragma unroll
-            for (int m = 0; m < 4; ++m)
-                v[m] = tt + m < L ? __bfloat162float(prm.dt[((long long)b * L + tt + m) * prm.H + h]) * a : 0.f;
-            v[1] += v[0];
-            v[2] += v[1];
-            v[3] += v[2];
-            float incl = v[3];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float u = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += u;
-            }
-            const float excl = incl - v[3] + pre;
-#pragma unroll
-            for (int m = 0; m < 4; ++m) cum[warp * kBlk + 4 * lane + m] = expf(excl + v[m]);
-        }
-        if (tid == 0) {  // the MMAs of block i (the accumulator was read out by block i - 1's epilogue)
-            if (wait_phase(&ld_bar[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag, status)) {
+    if (warp == 8) {
+        // ------------------------------------------------------------- producer (one thread)
+        if (lane == 0) {
+            int last_mma = -1, last_ld = -1;
+            bool ok = true;
+            auto store = [&](int i) {  // y tiles of block i, once the epilogue has updated them
+                ok = wait_phase(&y_done[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag, status);
+                if (!ok) return;
+                const int t0 = (blk0 + i) * kBlk;
+                for (int hh = 0; hh < 2; ++hh)
+                    tma_store_4d(&tm_y, y_tile + ((i & 1) * 2 + hh) * kPanel, 0, h0 + hh, t0, b, policy_evict_first());
+                bulk_commit();
+            };
+            for (int i = 0; i < nb && ok; ++i) {
+                // C is free once block i-1's MMAs are done, y buffer i % 2 once block i-2's store has
+                // read it (every store committed so far)
+                if (i >= 1 && !(ok = wait_phase(&mma_bar[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u, abort_flag, status)))
+                    break;
+                if (i >= 2) bulk_wait_read();
+                {
+                    const int t0 = (blk0 + i) * kBlk;
+                    uint64_t *bar = &ld_bar[i & 1];
+                    mbar_arrive_tx(bar, load_bytes);
+                    for (int pn = 0; pn < npan; ++pn) tma_load_4d(c_tile + pn * kPanel, &tm_c, bar, 64 * pn, g, t0, b);
+                    for (int e = 0; e < 2; ++e)
+                        tma_load_4d(y_tile + ((i & 1) * 2 + e) * kPanel, &tm_y, bar, 0, h0 + e, t0, b);
+                    last_ld = i;
+                }
+                // block i's MMAs into accumulator i % 2 (read out by block i-2's epilogue) while the
+                // epilogue works on block i-1
+                if (!(ok = wait_phase(&ld_bar[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag, status))) break;
+                if (i >= 2 && !(ok = wait_phase(&acc_free[i & 1], (uint32_t)((i - 2) >> 1) & 1u, abort_flag, status)))
+                    break;
                 tc_fence_after();
                 const uint32_t ca = smem_u32(c_tile), sa = smem_u32(s_tile);
                 constexpr uint32_t kId = idesc(128, 128, false, false);
 #pragma unroll 1
                 for (int kk = 0; kk < N / 16; ++kk) {
                     const uint32_t off = (uint32_t)((kk >> 2) * kPanel + (kk & 3) * 32);
-                    mma_ss(tmem, sdesc(ca + off, 16, 1024), sdesc(sa + off, 16, 1024), kId, kk > 0);
+                    mma_ss(tmem + 128 * (i & 1), sdesc(ca + off, 16, 1024), sdesc(sa + off, 16, 1024), kId, kk > 0);
                 }
-                mma_commit(mma_bar);
+                mma_commit(&mma_bar[i & 1]);
                 last_mma = i;
+                if (i >= 1) store(i - 1);  // block i-1's y tiles, once the epilogue has updated them
+            }
+            if (ok && nb > 0) store(nb - 1);
+            bulk_wait_all();
+            if (!ok) {  // MMAs and loads still in flight end before TMEM and the CTA go
+                const unsigned long long w0 = now_ns();
+                while (last_mma >= 0 && !mbar_try(&mma_bar[last_mma & 1], (uint32_t)(last_mma >> 1) & 1u) &&
+                       now_ns() - w0 < kWaitNs) {
+                }
+                while (last_ld >= 0 && !mbar_try(&ld_bar[last_ld & 1], (uint32_t)(last_ld >> 1) & 1u) &&
+                       now_ns() - w0 < 2 * kWaitNs) {
+                }
             }
         }
-        ok = wait_warp(mma_bar, (uint32_t)i & 1u, abort_flag, status) &&
-             wait_warp(&ld_bar[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag, status);
-        ok = __syncthreads_and(ok);
-        if (!ok) break;
-        tc_fence_after();
-        // C is free once the MMAs are done, and y buffer (i + 1) % 2 once the store of block i - 1
-        // has read it: the next block's tiles load during this block's epilogue
-        if (tid == 0 && i + 1 < nb) {
-            bulk_wait_read();
-            issue_loads(i + 1);
-            last_ld = i + 1;
-        }
-        {
-            const float w = cum[e * kBlk + row];
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------- epilogue (warps 0-7)
+        const int q = warp & 3, e = warp >> 2, row = 32 * q + lane;  // TMEM lane quarter, head
+        for (int i = 0; i < nb; ++i) {
+            const int blk = blk0 + i;
+            const long long t0 = (long long)blk * kBlk;
+            float *ck = cum + (i & 1) * 2 * kBlk;  // (two buffers: warps 0-1 may run one block ahead)
+            if (warp < 2) {  // decay factors exp(cumulative dt A) of head h0 + warp over the block's tokens
+                const int h = h0 + warp;
+                const float a = prm.A[h];
+                const float *bs = prm.bsum + ((long long)b * prm.H + h) * prm.nblk;
+                float pre = 0.f;
+                for (int k = lane; k < blk; k += 32) pre += bs[k];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) pre += __shfl_xor_sync(0xffffffffu, pre, o);
+                const long long tt = t0 + 4 * lane;
+                float v[4];
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    v[m] = tt + m < L ? __bfloat162float(prm.dt[((long long)b * L + tt + m) * prm.H + h]) * a : 0.f;
+                v[1] += v[0];
+                v[2] += v[1];
+                v[3] += v[2];
+                float incl = v[3];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float u = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += u;
+                }
+                const float excl = incl - v[3] + pre;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) ck[warp * kBlk + 4 * lane + m] = expf(excl + v[m]);
+            }
+            // (a wait that runs out raises the abort flag before the barrier, so after it every
+            // epilogue warp takes the same branch)
+            // (the y tiles' landing is awaited too: that is what makes their bytes visible here)
+            if (wait_phase(&ld_bar[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag, status))
+                wait_phase(&mma_bar[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag, status);
+            asm volatile("bar.sync 1, %0;" ::"n"(kEpi) : "memory");  // cum of this block written
+            if (*abort_flag) break;
+            tc_fence_after();
+            const float w = ck[e * kBlk + row];
+            const uint32_t taddr = tmem + 128 * (i & 1) + ((uint32_t)(32 * q) << 16) + 64 * e;
             unsigned char *yr = y_tile + ((i & 1) * 2 + e) * kPanel;
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
                 uint32_t acc[32];
                 tmem_ld32(taddr + 32 * half, acc);
                 tmem_wait_ld(acc);
+                if (half == 1) {
+                    tc_fence_before();
+                    mbar_arrive(&acc_free[i & 1]);
+                }
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {  // 16-byte chunks 4 half + c4 of the row (8 columns each)
                     uint4 *pv = reinterpret_cast<uint4 *>(yr + swz(row, 4 * half + c4));
@@ -205,29 +250,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     *pv = make_uint4(nv[0], nv[1], nv[2], nv[3]);
                 }
             }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();  // y tiles written, accumulator and cum read out
-        if (tid == 0) {
-            for (int hh = 0; hh < 2; ++hh)
-                tma_store_4d(&tm_y, y_tile + ((i & 1) * 2 + hh) * kPanel, 0, h0 + hh, (int)t0, b, policy_evict_first());
-            bulk_commit();
+            fence_proxy_async();
+            mbar_arrive(&y_done[i & 1]);
         }
     }
-    if (tid == 0) bulk_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
     if (warp == 0) {
-        if (lane == 0 && !ok) {  // MMAs and loads still in flight end before TMEM and the CTA go
-            const unsigned long long w0 = now_ns();
-            while (last_mma >= 0 && !mbar_try(mma_bar, (uint32_t)last_mma & 1u) && now_ns() - w0 < kWaitNs) {
-            }
-            while (last_ld >= 0 && !mbar_try(&ld_bar[last_ld & 1], (uint32_t)(last_ld >> 1) & 1u) &&
-                   now_ns() - w0 < 2 * kWaitNs) {
-            }
-        }
         __syncwarp();
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256) : "memory");
     }
 }
 
@@ -259,10 +291,12 @@ cudaError_t cp_correct_tc_launch(const CpProblem &p, const void *dt, const float
     prm.N = (int)p.N;
     prm.nblk = nblk;
     prm.pairs_per_group = (int)(p.H / p.G / 2);
-    // about one CTA per SM: each takes a run of consecutive blocks of one (batch row, head pair)
-    const long long tiles = (long long)nblk * p.G * prm.pairs_per_group * p.B;
+    // at most one CTA per SM (one wave): each takes a run of consecutive blocks of one (batch
+    // row, head pair); with more pairs than SMs, a whole stream each
+    const long long pairs = p.G * prm.pairs_per_group * p.B;
     const int sms = tc::num_sms() > 0 ? tc::num_sms() : 148;
-    prm.blocks_per_cta = (int)std::max(1ll, std::min((long long)nblk, (tiles + sms - 1) / sms));
+    const long long per_pair = std::max(1ll, (long long)sms / pairs);  // CTAs per pair
+    prm.blocks_per_cta = (int)std::max(1ll, ((long long)nblk + per_pair - 1) / per_pair);
     const int smem = smem_bytes((int)p.N) + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_correct_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
