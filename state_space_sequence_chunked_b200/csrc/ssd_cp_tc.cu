@@ -10,10 +10,11 @@
 // of consecutive 128-token blocks, all of which share S_in, and pipelines them:
 //   - the 8 epilogue warps first write S_in once, converted to bf16, K-major with 128-byte
 //     swizzle;
-//   - warp 8 (one thread) loads each block's C (one buffer: it is free once the block's MMAs
-//     are done) and the two heads' y tiles (two buffers), issues the block's dstate / 16 MMAs
-//     (M = 128, N = 128) into one of two TMEM accumulators, and stores each block's y tiles
-//     once the epilogue has updated them, so block i+1's loads and MMAs run during block i's
+//   - warp 8 (one thread) loads each block's C panel by panel into one buffer (a panel is
+//     reloaded for the next block as soon as this block's MMAs on it are done) and the two
+//     heads' y tiles (two buffers), issues the block's dstate / 16 MMAs (M = 128, N = 128),
+//     panel by panel, into one of two TMEM accumulators, and stores each block's y tiles once
+//     the epilogue has updated them, so block i+1's loads and MMAs run during block i's
 //     epilogue;
 //   - in the epilogue, warps 0-1 form the decay factors of the two heads; each warp reads its
 //     TMEM lane quarter for one head and updates the y tile in shared memory.
@@ -43,9 +44,9 @@ struct Params {
 };
 
 // Shared memory (after 1024-byte alignment): S_in tile [N/64 panels], C tile [N/64 panels],
-// y tiles [2 buffers][2 heads][128 rows x 128 B], cum [2 buffers][2 heads][128] fp32, 8 barriers,
+// y tiles [2 buffers][2 heads][128 rows x 128 B], cum [2 buffers][2 heads][128] fp32, 16 barriers,
 // TMEM base, abort flag and wait limit.
-__host__ __device__ constexpr int smem_bytes(int N) { return 2 * (N / 64) * kPanel + 4 * kPanel + 4 * kBlk * 4 + 128; }
+__host__ __device__ constexpr int smem_bytes(int N) { return 2 * (N / 64) * kPanel + 4 * kPanel + 4 * kBlk * 4 + 192; }
 
 __global__ void __launch_bounds__(kThreads, 1)
     k_correct_tc(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y, const Params prm) {
@@ -57,11 +58,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char *c_tile = sm + npan * kPanel;
     unsigned char *y_tile = sm + 2 * npan * kPanel;  // [2][2][16 KB]
     float *cum = reinterpret_cast<float *>(y_tile + 4 * kPanel);       // [2][2][128]
-    uint64_t *ld_bar = reinterpret_cast<uint64_t *>(cum + 4 * kBlk);  // [2] C and y tiles of block i landed (i % 2)
-    uint64_t *mma_bar = ld_bar + 2;    // [2] the MMAs of block i done (accumulator i % 2)
-    uint64_t *acc_free = ld_bar + 4;   // [2] accumulator i % 2 read out by the epilogue
-    uint64_t *y_done = ld_bar + 6;     // [2] y tiles of buffer i % 2 updated by the epilogue
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ld_bar + 8);
+    uint64_t *c_full = reinterpret_cast<uint64_t *>(cum + 4 * kBlk);  // [4] C panel p of the block landed
+    uint64_t *c_free = c_full + 4;     // [4] the block's MMAs on C panel p done
+    uint64_t *ld_bar = c_full + 8;     // [2] y tiles of block i landed (buffer i % 2)
+    uint64_t *mma_bar = c_full + 10;   // [2] the MMAs of block i done (accumulator i % 2)
+    uint64_t *acc_free = c_full + 12;  // [2] accumulator i % 2 read out by the epilogue
+    uint64_t *y_done = c_full + 14;    // [2] y tiles of buffer i % 2 updated by the epilogue
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c_full + 16);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int local_status = 0;
     int *status = prm.status ? prm.status : &local_status;
@@ -74,6 +77,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long L = prm.L;
 
     if (tid == 0) {
+        for (int p = 0; p < 4; ++p) {
+            mbar_init(&c_full[p], 1);
+            mbar_init(&c_free[p], 1);
+        }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&ld_bar[i], 1);
             mbar_init(&mma_bar[i], 1);
@@ -94,7 +101,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t load_bytes = (uint32_t)(npan * kPanel + 2 * kPanel);
 
     if (warp < 8) {
         // S_in of the two heads -> bf16, K-major: row r = 64 e + p, 16-byte chunk (n / 8) in panel
@@ -128,8 +134,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 8) {
         // ------------------------------------------------------------- producer (one thread)
         if (lane == 0) {
-            int last_mma = -1, last_ld = -1;
+            int last_mma = -1, last_c = -1, last_y[2] = {-1, -1};
             bool ok = true;
+            auto load_c = [&](int i, int pn) {  // C panel pn of block i
+                mbar_arrive_tx(&c_full[pn], kPanel);
+                tma_load_4d(c_tile + pn * kPanel, &tm_c, &c_full[pn], 64 * pn, g, (blk0 + i) * kBlk, b);
+            };
+            auto load_y = [&](int i) {  // the two heads' y tiles of block i, into buffer i % 2
+                mbar_arrive_tx(&ld_bar[i & 1], 2 * kPanel);
+                for (int e = 0; e < 2; ++e)
+                    tma_load_4d(y_tile + ((i & 1) * 2 + e) * kPanel, &tm_y, &ld_bar[i & 1], 0, h0 + e, (blk0 + i) * kBlk, b);
+                last_y[i & 1] = i;
+            };
             auto store = [&](int i) {  // y tiles of block i, once the epilogue has updated them
                 ok = wait_phase(&y_done[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag, status);
                 if (!ok) return;
@@ -138,37 +154,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_store_4d(&tm_y, y_tile + ((i & 1) * 2 + hh) * kPanel, 0, h0 + hh, t0, b, policy_evict_first());
                 bulk_commit();
             };
+            if (nb > 0) {
+                for (int pn = 0; pn < npan; ++pn) load_c(0, pn);
+                last_c = 0;
+                load_y(0);
+                if (nb > 1) load_y(1);
+            }
             for (int i = 0; i < nb && ok; ++i) {
-                // C is free once block i-1's MMAs are done, y buffer i % 2 once block i-2's store has
-                // read it (every store committed so far)
-                if (i >= 1 && !(ok = wait_phase(&mma_bar[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u, abort_flag, status)))
-                    break;
-                if (i >= 2) bulk_wait_read();
-                {
-                    const int t0 = (blk0 + i) * kBlk;
-                    uint64_t *bar = &ld_bar[i & 1];
-                    mbar_arrive_tx(bar, load_bytes);
-                    for (int pn = 0; pn < npan; ++pn) tma_load_4d(c_tile + pn * kPanel, &tm_c, bar, 64 * pn, g, t0, b);
-                    for (int e = 0; e < 2; ++e)
-                        tma_load_4d(y_tile + ((i & 1) * 2 + e) * kPanel, &tm_y, bar, 0, h0 + e, t0, b);
-                    last_ld = i;
-                }
-                // block i's MMAs into accumulator i % 2 (read out by block i-2's epilogue) while the
-                // epilogue works on block i-1
-                if (!(ok = wait_phase(&ld_bar[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag, status))) break;
+                // block i's MMAs, panel by panel, into accumulator i % 2 (read out by block i-2's
+                // epilogue) while the epilogue works on block i-1
                 if (i >= 2 && !(ok = wait_phase(&acc_free[i & 1], (uint32_t)((i - 2) >> 1) & 1u, abort_flag, status)))
                     break;
-                tc_fence_after();
-                const uint32_t ca = smem_u32(c_tile), sa = smem_u32(s_tile);
                 constexpr uint32_t kId = idesc(128, 128, false, false);
-#pragma unroll 1
-                for (int kk = 0; kk < N / 16; ++kk) {
-                    const uint32_t off = (uint32_t)((kk >> 2) * kPanel + (kk & 3) * 32);
-                    mma_ss(tmem + 128 * (i & 1), sdesc(ca + off, 16, 1024), sdesc(sa + off, 16, 1024), kId, kk > 0);
+                const uint32_t ca = smem_u32(c_tile), sa = smem_u32(s_tile);
+                for (int pn = 0; pn < npan && ok; ++pn) {
+                    if (!(ok = wait_phase(&c_full[pn], (uint32_t)i & 1u, abort_flag, status))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const uint32_t off = (uint32_t)(pn * kPanel + k4 * 32);
+                        mma_ss(tmem + 128 * (i & 1), sdesc(ca + off, 16, 1024), sdesc(sa + off, 16, 1024), kId,
+                               pn > 0 || k4 > 0);
+                    }
+                    mma_commit(&c_free[pn]);
                 }
+                if (!ok) break;
                 mma_commit(&mma_bar[i & 1]);
                 last_mma = i;
-                if (i >= 1) store(i - 1);  // block i-1's y tiles, once the epilogue has updated them
+                // block i+1's C, each panel as soon as this block's MMAs on it are done
+                if (i + 1 < nb) {
+                    for (int pn = 0; pn < npan && ok; ++pn) {
+                        if (!(ok = wait_phase(&c_free[pn], (uint32_t)i & 1u, abort_flag, status))) break;
+                        load_c(i + 1, pn);
+                    }
+                    if (!ok) break;
+                    last_c = i + 1;
+                }
+                // block i-1's y tiles out, then block i+1's in once that store has read its buffer
+                if (i >= 1) {
+                    store(i - 1);
+                    if (!ok) break;
+                    if (i + 1 < nb) {
+                        bulk_wait_read();
+                        load_y(i + 1);
+                    }
+                }
             }
             if (ok && nb > 0) store(nb - 1);
             bulk_wait_all();
@@ -177,9 +207,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 while (last_mma >= 0 && !mbar_try(&mma_bar[last_mma & 1], (uint32_t)(last_mma >> 1) & 1u) &&
                        now_ns() - w0 < kWaitNs) {
                 }
-                while (last_ld >= 0 && !mbar_try(&ld_bar[last_ld & 1], (uint32_t)(last_ld >> 1) & 1u) &&
-                       now_ns() - w0 < 2 * kWaitNs) {
-                }
+                for (int pn = 0; pn < npan && last_c >= 0; ++pn)
+                    while (!mbar_try(&c_full[pn], (uint32_t)last_c & 1u) && now_ns() - w0 < 2 * kWaitNs) {
+                    }
+                for (int k = 0; k < 2; ++k)
+                    while (last_y[k] >= 0 && !mbar_try(&ld_bar[k], (uint32_t)(last_y[k] >> 1) & 1u) &&
+                           now_ns() - w0 < 2 * kWaitNs) {
+                    }
             }
         }
         __syncwarp();
