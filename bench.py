@@ -47,18 +47,26 @@ def tc_kernel(wl):
     return "k_ssd_pair" if wl.dstate == 128 and (wl.nheads // wl.ngroups) % 2 == 0 else "k_ssd_tc<%d>" % wl.dstate
 
 
+def code_sha256(path):
+    """SHA-256 of a C++/CUDA source with its // comments and all whitespace removed: what the
+    compiler turns into code. (None of the kernel sources uses // inside a string literal.)"""
+    import hashlib
+    import re
+
+    text = open(path, encoding="utf-8").read()
+    code = "".join("".join(re.sub(r"//.*", "", line).split()) for line in text.splitlines())
+    return hashlib.sha256(code.encode()).hexdigest()
+
+
 def measured_traffic(wl, path):
     """DRAM bytes (read + write) per launch of the tensor-core kernel from the committed ncu
-    capture, if that capture was taken of the kernel source as it is now; else None."""
-    import hashlib
-
+    capture, if that capture was taken of the kernel's code as it is now; else None."""
     from state_space_sequence_chunked_b200 import inputs
 
     if wl != inputs.WORKLOADS["mamba2_2p7b"] or path != "tcgen05" or not os.path.exists(TRAFFIC_FILE):
         return None
     rec = json.load(open(TRAFFIC_FILE))
-    src = hashlib.sha256(open(TC_SOURCE, "rb").read()).hexdigest()
-    if rec.get("source_sha256") != src:
+    if rec.get("source_code_sha256") != code_sha256(TC_SOURCE):
         return None
     return rec["dram_read_bytes"] + rec["dram_write_bytes"]
 

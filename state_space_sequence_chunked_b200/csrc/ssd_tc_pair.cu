@@ -16,37 +16,42 @@
 // The running state stays in TMEM, in the chunk-state accumulator itself: before the chunk-
 // state product of block t the accumulator holds (gamma_t / dsc_t) S_t (gamma_t = exp(A_cs[127]),
 // dsc_t the factor of dS above), the product adds dS_t, and the result is S_{t+1} / dsc_t.
-// Between the two products one pass over the accumulator (E warps) recovers S_{t+1}, writes
+// Between the two products one pass over the accumulator (the S warps) recovers S_{t+1}, writes
 // its bf16 copy for step 4 of block t+1 and rescales the accumulator for block t+1.
 //
 // A block is factored for a head when its A_cs range is at most 192 (log2 units) and every
 // valid token has |dt| >= 2^-40. The row and column factors then stay within 2^+-96, which
 // leaves 2^31 of the exponent range that fp32 and bf16 share (up to 2^127) for |dt x| and the
 // 128-term sums of the products; a decay factor below 2^-126 flushes to 0, as the true value
-// is negligible next to the terms it is added to. A pair task in which either head's block is not factored is
-// run as two single-head tasks, each in the elementwise (exact) form for its head e, with
-// N = 64 products on that head's columns only:
-//   x_e stays in its half of the x slot; X'_e[s] = exp(A_cs_e[127] - A_cs_e[s]) dt_s x_s goes
-//   into the other half and feeds the chunk state; G'_e[l,s] = G[l,s] exp(A_cs_e[l] -
-//   A_cs_e[s]) dt_s (+ D_e on the diagonal) multiplies x_e; the rows of C are scaled by
-//   exp(A_cs_e[l]) in place; S_e enters unscaled and y_e = Y_e. The other head's state is kept.
+// is negligible next to the terms it is added to. A pair task in which either head's block is
+// not factored runs as two single-head tasks in the exact form of head e, with N = 64 products
+// on that head's columns only, factored by quarters of 32 tokens (mid_q the middle of quarter
+// q's A_cs span):
+//   X'''_e[s] = exp(mid_q(s) - A_cs_e[s]) dt_s x_s goes into the other head's half of the x slot
+//   (x_e stays in its own half); G'_e[l,s] = G[l,s] exp(A_cs_e[l] - mid_q(s)) for s <= l (one
+//   exp per row and quarter; element by element when a quarter spans more than 224); the other
+//   head's X warps scale B's rows by exp(A_cs_e[127] - A_cs_e[s]) dt_s in place once C B^T has
+//   read B, so the chunk state is B'^T x_e; the rows of C are scaled by exp(A_cs_e[l]) in place;
+//   S_e enters unscaled and y_e = Y_e + D_e x_e. The other head's state is kept.
 //
 // Work split, cut streams and the hand-over are those of the one-head kernel, over pair
 // streams (batch row, head pair): a persistent grid splits the pair tasks into equal shares;
 // a stream cut between two CTAs hands its state over through global memory (the state
 // passing of "序列并行" inside one GPU), ready long before it is read.
 //
-// Warp roles (1024 threads): warp 0 loads (TMA for C, B, x; dt with plain loads), runs step 0
-// over each block and decides its form; warps 1, 2, 3 each issue one product (C B^T; the
-// chunk states; Y); warps 4-7 ("T") write G' (and scale C in the exact form); warps 8-15 ("X",
-// 8 + 4 e + quarter for head e) write X'' of their head; warps 16-23 ("S", the same layout) run
-// its state pass; warps 24-31 ("O", the same layout) run the epilogue, staging y in the x slot
-// it came from. The jobs overlap: X'' of block t+1, the state pass of block t+1 and the
-// epilogue of block t run at the same time. Each
-// warp touches only the TMEM lane quarter of its warp index. Rings: C and B in two 64 KB stages, x in
-// two 32 KB slots, one S^T buffer; TMEM: two C B^T buffers, one state and one output
-// accumulator of 128 columns each. Every wait is bounded; on timeout the CTA raises bit 0 of
-// the status word, drains its own copies and MMAs, frees TMEM and returns.
+// Warp roles (1024 threads): warp 2 ("describer") fetches the dt of both heads one task ahead,
+// runs step 0 for both heads at once, decides the task's form, writes a descriptor into a ring
+// of four and issues the TMA loads of C and B; warp 0 loads x (each head's half as soon as its
+// previous y has left the slot) and prefetches the next task's x into L2; warp 1 issues C B^T
+// and the chunk states; warp 3 issues Y; warps 4-7 ("T") write G' (and scale C in the exact
+// form); warps 8-15 ("X", 8 + 4 e + quarter for head e) write X'' of their head (in the exact
+// form X''' or B's rows); warps 16-23 ("S", the same layout) run its state pass; warps 24-31
+// ("O", the same layout) run the epilogue, staging y in the x slot it came from. The jobs
+// overlap: X'' of block t+1, the state pass of block t+1 and the epilogue of block t run at the
+// same time. Each warp touches only the TMEM lane quarter of its warp index. Rings: C and B in
+// two 64 KB stages, x in two 32 KB slots, one S^T buffer; TMEM: two C B^T buffers, one state
+// and one output accumulator of 128 columns each. Every wait is bounded; on timeout the CTA
+// raises bit 0 of the status word, drains its own copies and MMAs, frees TMEM and returns.
 #include <algorithm>
 
 #include "tc_ptx.cuh"
