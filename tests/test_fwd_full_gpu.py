@@ -63,6 +63,17 @@ def test_every_stream_full_size(cuda_device, name):
     print(f"{name}: worst stream y {ey.max():.3e}, h_final {eh.max():.3e}")
 
 
+def cut_streams(nstreams, nblocks, sms):
+    """Streams split between two CTAs' shares, by the kernels' share rule: the stream-major
+    (stream, block) tasks cut into min(sms, nstreams) near-equal contiguous shares, share i
+    starting at task q i + (r i) // grid (q, r = divmod(total, grid))."""
+    grid = max(1, min(sms, nstreams))
+    total = nstreams * nblocks
+    q, r = divmod(total, grid)
+    starts = [q * i + (r * i) // grid for i in range(1, grid)]
+    return sorted({st // nblocks for st in starts if st % nblocks != 0})
+
+
 @pytest.mark.parametrize("dstate,nheads", [(128, 300), (256, 300), (128, 151), (256, 153)])
 def test_cut_streams_every_stream(cuda_device, dstate, nheads):
     """150 to 300 streams of 16 blocks over 148 CTAs: head pairs (300 heads at N = 128, the
@@ -73,4 +84,11 @@ def test_cut_streams_every_stream(cuda_device, dstate, nheads):
                              h0_std=0.2, seed=40 + dstate)
     d = inputs.draw(wl)
     assert plan_of(d, wl.chunk)["path"] == "tcgen05"
-    assert_every_stream(d, wl.chunk, cuda_device)
+    ey, eh = assert_every_stream(d, wl.chunk, cuda_device)
+    # the streams the share rule cuts, named explicitly (they are among those checked above)
+    pair = dstate == 128 and nheads % 2 == 0
+    sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
+    cut = cut_streams(wl.batch * (nheads // 2 if pair else nheads), wl.seqlen // 128, sms)
+    assert len(cut) > 100, len(cut)
+    heads = [h for c in cut for h in ((2 * c, 2 * c + 1) if pair else (c,))]
+    assert max(ey[0, heads]) <= TOL["bf16"] and max(eh[0, heads]) <= TOL["bf16"]
