@@ -90,11 +90,12 @@ def algorithmic(wl):
     return nbytes, flops
 
 
-def fwd_config(wl, path, l2):
-    """The config object of a forward line (both arms carry the same keys)."""
+def fwd_config(wl):
+    """The config object of a forward line: the workload alone, so both arms carry the same
+    keys and values (the path that ran is a separate key of the line)."""
     return {"workload": wl.name, "batch": wl.batch, "seqlen": wl.seqlen, "nheads": wl.nheads,
             "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk,
-            "dt": wl.dt_dist, "path": path, "per_rank_batch": wl.batch, "l2": l2}
+            "dt": wl.dt_dist, "per_rank_batch": wl.batch, "l2": l2_note(wl)}
 
 
 def l2_note(wl):
@@ -296,8 +297,7 @@ def reference_arm(args, wl):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * wl.batch * wl.seqlen / value, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": fwd_config(wl, "oracle: fp64 recurrence on the host cores",
-                             "n/a (host memory; the oracle streams the inputs from RAM)"),
+        "config": fwd_config(wl), "path": "oracle: fp64 recurrence on the host cores",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": f"fp64 recurrence on {n} of {wl.batch * wl.nheads} (batch, head) streams "
                                    f"over all {wl.seqlen} tokens per step, extrapolated to the whole batch"},
@@ -881,7 +881,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
-            "config": fwd_config(wl, plan["path"], l2_note(wl)),
+            "config": fwd_config(wl), "path": plan["path"],
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                          "frac": achieved / peak, "traffic": measured_traffic(wl, plan["path"]),
                          "kernel": ("%s (the whole call: one launch after a status-word memset)" % tc_kernel(wl)
