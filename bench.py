@@ -39,6 +39,7 @@ def peaks():
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "k_ssd_pair_mamba2_2p7b_traffic.json")
 TC_SOURCE = os.path.join(ROOT, "state_space_sequence_chunked_b200", "csrc", "ssd_tc_pair.cu")
+TC_HEADER = os.path.join(ROOT, "state_space_sequence_chunked_b200", "csrc", "tc_ptx.cuh")  # its inline PTX
 
 
 def tc_kernel(wl):
@@ -47,14 +48,16 @@ def tc_kernel(wl):
     return "k_ssd_pair" if wl.dstate == 128 and (wl.nheads // wl.ngroups) % 2 == 0 else "k_ssd_tc<%d>" % wl.dstate
 
 
-def code_sha256(path):
-    """SHA-256 of a C++/CUDA source with its // comments and all whitespace removed: what the
+def code_sha256(*paths):
+    """SHA-256 of C++/CUDA sources with their // comments and all whitespace removed: what the
     compiler turns into code. (None of the kernel sources uses // inside a string literal.)"""
     import hashlib
     import re
 
-    text = open(path, encoding="utf-8").read()
-    code = "".join("".join(re.sub(r"//.*", "", line).split()) for line in text.splitlines())
+    code = ""
+    for path in paths:
+        text = open(path, encoding="utf-8").read()
+        code += "".join("".join(re.sub(r"//.*", "", line).split()) for line in text.splitlines())
     return hashlib.sha256(code.encode()).hexdigest()
 
 
@@ -66,7 +69,7 @@ def measured_traffic(wl, path):
     if wl != inputs.WORKLOADS["mamba2_2p7b"] or path != "tcgen05" or not os.path.exists(TRAFFIC_FILE):
         return None
     rec = json.load(open(TRAFFIC_FILE))
-    if rec.get("source_code_sha256") != code_sha256(TC_SOURCE):
+    if rec.get("source_code_sha256") != code_sha256(TC_SOURCE, TC_HEADER):
         return None
     return rec["dram_read_bytes"] + rec["dram_write_bytes"]
 
