@@ -123,3 +123,54 @@ def test_mixer_reduces_to_pieces():
     want = oracle.gated_rmsnorm(y.reshape(1, L, HP), z, nw, ngroups=1, eps=1e-6)
     np.testing.assert_allclose(out, want, rtol=1e-13)
     np.testing.assert_allclose(hf, hf2, rtol=1e-13)
+
+
+def test_mixer_one_token_closed_form():
+    """One token from a zero state, with random projections, written out by hand: the causal
+    convolution sees only its last tap, the state is dt x B^T, y = dt (B . C) x + D x, then the
+    gate, the grouped norm and the output projection. Pins the column order of the input
+    projection's row, the tap alignment, the step-size map and the order of the steps."""
+    rng = np.random.default_rng(11)
+    H, P, G, N, W, dm = 4, 2, 2, 3, 4, 5
+    HP, GN = H * P, G * N
+    Dp = 2 * HP + 2 * GN + H
+    u = rng.standard_normal((1, 1, dm))
+    in_w = rng.standard_normal((Dp, dm)) * 0.4
+    out_w = rng.standard_normal((dm, HP)) * 0.4
+    conv_w = rng.standard_normal((HP + 2 * GN, W)) * 0.5
+    conv_b = rng.standard_normal(HP + 2 * GN) * 0.1
+    dtb = rng.uniform(-2.0, 0.0, H)
+    A, D = -rng.uniform(0.5, 3.0, H), rng.standard_normal(H)
+    nw = 1.0 + 0.1 * rng.standard_normal(HP)
+    eps = 1e-6
+    out, hf = oracle.mamba2_mixer(u, in_w, conv_w, conv_b, dtb, A, D, nw, out_w, nheads=H, headdim=P, ngroups=G,
+                                  dstate=N, norm_groups=2, eps=eps)
+
+    row = [sum(in_w[c, k] * u[0, 0, k] for k in range(dm)) for c in range(Dp)]
+    z = row[:HP]
+    act = [0.0] * (HP + 2 * GN)
+    for c in range(HP + 2 * GN):
+        v = conv_w[c, W - 1] * row[HP + c] + conv_b[c]  # only the newest tap sees a token
+        act[c] = v / (1.0 + math.exp(-v))
+    xs, Bs, Cs = act[:HP], act[HP:HP + GN], act[HP + GN:]
+    y = [0.0] * HP
+    state = np.zeros((H, P, N))
+    for h in range(H):
+        dt = math.log1p(math.exp(row[2 * HP + 2 * GN + h] + dtb[h]))
+        g = h // (H // G)
+        bc = sum(Bs[g * N + n] * Cs[g * N + n] for n in range(N))
+        for p in range(P):
+            xv = xs[h * P + p]
+            y[h * P + p] = dt * bc * xv + D[h] * xv
+            for n in range(N):
+                state[h, p, n] = dt * xv * Bs[g * N + n]
+    gated = [y[c] * z[c] / (1.0 + math.exp(-z[c])) for c in range(HP)]
+    normed = [0.0] * HP
+    gs = HP // 2
+    for k in range(2):
+        ms = sum(gated[c] ** 2 for c in range(k * gs, (k + 1) * gs)) / gs
+        for c in range(k * gs, (k + 1) * gs):
+            normed[c] = nw[c] * gated[c] / math.sqrt(ms + eps)
+    want = [sum(out_w[j, c] * normed[c] for c in range(HP)) for j in range(dm)]
+    np.testing.assert_allclose(out[0, 0], want, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(hf[0], state, rtol=1e-12, atol=1e-15)
