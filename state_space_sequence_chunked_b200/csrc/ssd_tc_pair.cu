@@ -142,7 +142,7 @@ __device__ __forceinline__ float quarter_cumsum(float dt, float a2, float off, i
     return __fadd_rn(off, incl);
 }
 
-// Per head and task, written by the load warp next to the task's dt: the middle m of the
+// Per head and task, written by the describer warp next to the task's dt: the middle m of the
 // block's A_cs range, the block total, the cumsum at the end of quarters 0, 1, 2, A_h log2(e)
 // and D_h (0 without D).
 struct Head0 {
@@ -258,14 +258,12 @@ __device__ __forceinline__ uint32_t ld_dt_pair(const __nv_bfloat16 *p, uint64_t 
     return v;
 }
 
-// Per (task, head) factors of the state pass: gamma = exp(A_cs[127]), dsc = the chunk state's
-// factor (exp(A_cs[127] - m) factored, 1 exact), sg = the scale of the bf16 copy (exp(m)
-// factored, 1 exact); a head that is not in a single-head task keeps its state: all 1.
-// Per head and block: dsc scales the block's chunk-state product (the accumulator then holds
-// S_{t+1} / dsc), sg the bf16 copy of the state for the state-to-output product, rs the state
-// the accumulator holds before the product ((gamma / dsc) S, gamma = exp(A_cs[127])). In the
-// factored form sg = rs = exp(m) exactly; in the exact form of the head the state enters
-// unscaled (sg = 1) and the accumulator holds gamma S; the other head's state passes through.
+// Per head and block, the factors of the state pass (gamma = exp(A_cs[127])): dsc scales the
+// block's chunk-state product (the accumulator then holds S_{t+1} / dsc), sg the bf16 copy of
+// the state for the state-to-output product, rs the state the accumulator holds before the
+// product ((gamma / dsc) S). Factored: dsc = exp(A_cs[127] - m), sg = rs = exp(m). The head of
+// a single-head (exact) task: dsc = sg = 1, rs = gamma (its state enters unscaled). The other
+// head of a single-head task keeps its state: all 1.
 struct StateF {
     float dsc, sg, rs;
 };
@@ -554,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float dv = (i & 1) ? bf16_hi(hv[i >> 1]) : bf16_lo(hv[i >> 1]);
                 dt_ok = dt_ok && (nv <= i || fabsf(dv) >= 0x1p-40f);
             }
-            // (mx - mn <= 128 is false for NaN, which then takes the exact form)
+            // (mx - mn <= 192 is false for NaN, which then takes the exact form)
             const bool fact = __all_sync(0xffffffffu, dt_ok && (mx - mn <= 192.f));
             // Head0 = {m, tot, off1, off2, off3, a2, Dh, 0}; off q = the cumsum through token 32 q - 1;
             // lane 16 e + f (f < 8) holds field f of head e
@@ -792,10 +790,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!wait_warp(&gfull[j], (uint32_t)(t >> 1) & 1u, abort_flag, status)) break;
             tc_fence_after();
             if (mode == kModePair) {
-                // 16-column pieces: below the diagonal a plain conversion to bf16 pairs; the piece
-                // holding the diagonal masks s > row; above it zeros
-                // 32 columns (two 16-column pieces) per load: the pieces of block jb <= qtr hold
-                // this warp's rows' causal part, those above are zeros
+                // 32 columns per load, 16 packed bf16 pair columns per store: blocks jb < qtr are
+                // converted as they are, the diagonal block jb == qtr masks s > row, blocks above
+                // it are zeros
 #pragma unroll 1
                 for (int jb = 0; jb < 4; ++jb) {
                     uint32_t out[16];
@@ -829,7 +826,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&gp[j]);
         }
     } else if (warp < kWarpS) {
-        // ------------------------------------------------------------- X: X'' (factored) or X' (exact) of head e
+        // ------------------------------------------------------------- X: X'' (factored) of head e, or in the exact form X''' or B's rows
         const int qtr = warp & 3, e = (warp - kWarpX) >> 2;
         const int row = (qtr << 5) | lane;
         for (int t = 0;; ++t) {
