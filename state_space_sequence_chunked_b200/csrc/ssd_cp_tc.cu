@@ -28,7 +28,7 @@ namespace ssd {
 namespace cpt {
 using namespace tc;
 
-constexpr int kBlk = 128;      // tokens per CTA
+constexpr int kBlk = 128;      // tokens per block
 constexpr int kP = 64;         // head dimension this kernel takes
 constexpr int kPanel = 16384;  // one 64-column panel of a 128-row K-major tile, bytes
 constexpr int kThreads = 288;  // 8 epilogue warps and the producer warp

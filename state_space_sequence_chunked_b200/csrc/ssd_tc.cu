@@ -1,7 +1,7 @@
 // Fused chunked SSD forward on 5th-generation tensor cores (tcgen05, sm_100a).
 //
-// A persistent grid (one CTA per SM) splits the B*H*nc (stream, 128-token block)
-// tasks into equal contiguous shares; within a share each stream's blocks are
+// A persistent grid (one CTA per SM, or one per stream when there are fewer streams)
+// splits the B*H*nc (stream, 128-token block) tasks into equal contiguous shares; within a share each stream's blocks are
 // walked in order, so x is read once, y is written once and the running state
 // stays on chip. Per block (the four steps of "SSD 算法：分块和状态传递" in the
 // Mamba-2 SSD write-up, with the block decomposition of "SSD 算法：分块矩阵分解"):
@@ -33,11 +33,12 @@
 // CTA holding the rest runs it last, so the hand-over is ready long before it is
 // read. The wait for it is bounded all the same.
 //
-// Warp roles (384 threads): warp 0 loads (TMA + dt) and runs step 0; warps 1, 2 and 3
-// issue C B^T, the chunk states and Y (one issuing thread per product: an MMA
-// instruction keeps its issuing warp busy for ~100 cycles, so the products are issued
-// in parallel); warps 4-7 ("T") do X'' and G'; warps 8-11 ("E") run the state chain and
-// the epilogue. B and C, and x with its step-0 values, have separate stage barriers, so
+// Warp roles (384 threads at N = 128, 512 at N = 256): warp 0 loads (TMA + dt) and runs
+// step 0; warps 1, 2 and 3 issue C B^T, the chunk states and Y (one issuing thread per
+// product: an MMA instruction keeps its issuing warp busy for ~100 cycles, so the products
+// are issued in parallel); warps 4-7 ("T") do X'' and G'; warps 8-11 ("E"), and 12-15 at
+// N = 256, run the state chain, one set of four warps per 128 state rows, and the first set
+// runs the epilogue. B and C, and x with its step-0 values, have separate stage barriers, so
 // the next block's B and C load as soon as the products that read them are done. Every
 // wait is bounded: on timeout the CTA raises a status word in the workspace, drains its
 // own TMA loads and MMAs, frees TMEM and returns.
