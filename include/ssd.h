@@ -16,8 +16,10 @@
  *
  * Conventions for every entry point below:
  *  - All tensor pointers are DEVICE pointers owned by the caller, row-major and
- *    contiguous, 16-byte aligned. The library allocates no memory, keeps no global
- *    mutable state and may be called from several host threads at once.
+ *    contiguous, 16-byte aligned. The library allocates no memory and may be called
+ *    from several host threads at once. Its only global mutable state is the test
+ *    hook's wait limit (ssd_set_wait_limit_us) and the built-in device array of
+ *    ssd_fwd_static_scratch.
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *    stream). Calls are asynchronous: SSD_OK means "validated and launched".
  *    Faults inside a kernel surface from a later CUDA call or synchronisation.
